@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the DiT joint-attention hot path on B200.
+
+One step = one pass of the hot path over the Flux-like 2048-px workload
+(B=1, H=24, N=512 text + 128x128 image = 16896 tokens, d=128):
+rotary embedding of Q and K, BF16 joint attention, and the First-Block-Cache
+gate on a 16896 x 3072 bf16 hidden-state residual pair.  The FP8 variant
+(rotary + K smoothing + per-block e4m3 quantisation + FP8 attention) is timed
+the same way and reported in the "fp8" object.
+
+value = attention FLOPs (4*B*H*N^2*d per call) x calls / device time, in
+TFLOP/s, summed over ranks (each rank runs its own independent problem: weak
+scaling, no data-path collective).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DiT joint-attention TFLOP/s and % of B200 BF16/FP8 tensor peak, N=16896"
+WORKLOAD = "flux2k"
+HIDDEN = 3072
+THRESHOLD = 0.12
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel, keyed
+# by the hash of the kernel source it was taken on; a changed kernel reports null.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "diffusion_transformer_denoising_dit_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def aggregate(elapsed_ms_per_rank, units_per_rank, steps):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = max(elapsed_ms_per_rank)
+    total = sum(units_per_rank)
+    return total / (t / 1e3), t / steps
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------- CPU oracle legs
+def oracle_sample(q, k, v, pos, w, heads, rows):
+    """Exact fp64 attention of the oracle on `heads` heads x `rows` query rows. Returns (flops, seconds)."""
+    from oracle import attention as A
+    t0 = time.perf_counter()
+    A.attention(q[:, :heads], k[:, :heads], v[:, :heads], pos=pos, axes=w.axes, theta=w.theta,
+                rows=None if rows >= w.N else __import__("numpy").arange(rows))
+    dt = time.perf_counter() - t0
+    return 4.0 * heads * rows * w.N * w.d, dt
+
+
+def cpu_cores():
+    try:
+        import numpy  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("num_threads")]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step = one bounded sample of the workload on host cores."""
+    if rank != 0:
+        return
+    import torch
+    from diffusion_transformer_denoising_dit_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    q, k, v = synth.qkv(w)
+    pos = synth.positions(w.T, w.G).numpy()
+    rows = 512
+    for _ in range(args.warmup):
+        oracle_sample(q, k, v, pos, w, 1, rows)
+    flops, t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(q, k, v, pos, w, 1, rows)
+        flops += f
+        t += dt
+    val = flops / t / 1e12
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "flux2k B=1 H=24 N=16896 d=128, RoPE axes (16,56,56)",
+                                        "sample": f"1 head x {rows} query rows per step"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"fp64 exact attention with RoPE, 1 head x {rows} query rows x 16896 keys per step"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import diffusion_transformer_denoising_dit_b200 as dit
+    from diffusion_transformer_denoising_dit_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[WORKLOAD]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    flops = w.flops()
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    q, k, v = synth.qkv(w, device=dev, seed=w.seed + rank)
+    pos = synth.positions(w.T, w.G).to(dev)
+    cos, sin = dit.rope_tables(pos, w.axes, w.theta)
+    r_prev, r_cur = (t.contiguous() for t in synth.gate_pair(N, HIDDEN, 0.05, seed=4000 + rank, device=dev))
+    o = torch.empty_like(q)
+    ws = dit.attention_workspace(B, H, N, d, "bf16", rope=True, device=dev)
+    gate = dit.FBCacheGate(THRESHOLD, r_cur.numel(), device=dev)
+    have_fp8 = True
+    try:
+        ws8 = dit.attention_workspace(B, H, N, d, "fp8", device=dev)
+        dit.attention(q, k, v, cos, sin, precision="fp8", out=o, workspace=ws8)
+    except dit.DitError:
+        have_fp8 = False
+
+    def step_bf16():
+        dit.attention(q, k, v, cos, sin, out=o, workspace=ws)
+        gate(r_cur, r_prev)
+
+    def step_fp8():
+        dit.attention(q, k, v, cos, sin, precision="fp8", out=o, workspace=ws8)
+        gate(r_cur, r_prev)
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return [x]
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        out = [torch.zeros_like(t) for _ in range(world)]
+        dist.all_gather(out, t)
+        return [float(z.item()) for z in out]
+
+    # ---- main timed region: BF16 step (rotary + attention + gate)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        ms = timed(step_bf16, args.steps, args.warmup)
+    clocks = clk.summary()
+    all_ms = max_over_ranks(ms)
+    value, ms_per_step = aggregate(all_ms, [flops * args.steps] * world, args.steps)
+    assert dit.read_error() == 0
+
+    # ---- dominant kernel alone: attention on pre-rotated Q/K (exactly one attn launch)
+    qr = dit.rope_apply(q, cos, sin)
+    kr = dit.rope_apply(k, cos, sin)
+    ka = max(5, args.steps)
+    ms_attn = timed(lambda: dit.attention(qr, kr, v, out=o), ka, 3) / ka
+    achieved = flops / (ms_attn / 1e3) / 1e12
+    bf16_peak = peaks["bf16_tflops"]
+    h_attn = _src_hash("attn_bf16.cu", "dit_device.cuh")
+    tr = NCU_TRAFFIC.get(("attn_bf16", h_attn))
+    roofline = {"bound": "tensor", "kernel": "attn_bf16_kernel<128>", "achieved": achieved, "peak": bf16_peak,
+                "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": tr,
+                "peak_source": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
+                "frac_of_nominal_2250": achieved / 2250.0, "ms_per_launch": ms_attn}
+
+    # ---- side kernels alone: rotary pre-pass and the gate (HBM-bound)
+    kr2 = torch.empty_like(k)
+    ms_rope = timed(lambda: dit.rope_apply(k, cos, sin, out=kr2), ka, 3) / ka
+    rope_bytes = 2 * k.numel() * 2 + 2 * cos.numel() * 4
+    ms_gate = timed(lambda: gate(r_cur, r_prev), ka, 3) / ka
+    gate_bytes = 2 * r_cur.numel() * 2
+    hbm = peaks["hbm_gbs"]
+    side = {
+        "rope_apply": {"GB/s": rope_bytes / (ms_rope / 1e3) / 1e9, "frac": rope_bytes / (ms_rope / 1e3) / 1e9 / hbm,
+                       "ms": ms_rope, "bytes": rope_bytes},
+        "fbcache_gate": {"GB/s": gate_bytes / (ms_gate / 1e3) / 1e9,
+                         "frac": gate_bytes / (ms_gate / 1e3) / 1e9 / hbm, "ms": ms_gate, "bytes": gate_bytes},
+    }
+
+    # ---- FP8 step
+    fp8 = None
+    if have_fp8:
+        ms8 = timed(step_fp8, args.steps, args.warmup)
+        all8 = max_over_ranks(ms8)
+        v8, mps8 = aggregate(all8, [flops * args.steps] * world, args.steps)
+        fp8_peak = 2.0 * bf16_peak
+        fp8 = {"value": v8 / 1e12, "unit": "TFLOP/s", "ms_per_step": mps8,
+               "peak": fp8_peak, "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
+               "frac_of_step": v8 / 1e12 / fp8_peak}
+        assert dit.read_error() == 0
+
+    # ---- e2e through the public API from pinned host buffers
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hrc, hrp = r_cur.cpu().pin_memory(), r_prev.cpu().pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hskip = torch.empty(1, dtype=torch.int32).pin_memory()
+
+    def step_e2e():
+        dq, dk, dv = (t.to(dev, non_blocking=True) for t in (hq, hk, hv))
+        drc, drp = hrc.to(dev, non_blocking=True), hrp.to(dev, non_blocking=True)
+        out = dit.attention(dq, dk, dv, cos, sin, workspace=ws)
+        flag = gate(drc, drp)
+        ho.copy_(out, non_blocking=True)
+        hskip.copy_(flag, non_blocking=True)
+
+    ke = max(3, min(args.steps, 10))
+    ms_e2e = timed(step_e2e, ke, 2)
+    all_e2e = max_over_ranks(ms_e2e)
+    e2e_val, _ = aggregate(all_e2e, [flops * ke] * world, ke)
+    h2d = (q.numel() + k.numel() + v.numel() + r_cur.numel() + r_prev.numel()) * 2
+    d2h = o.numel() * 2 + 4
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        posn = pos.cpu().numpy()
+        f_tot, t_tot, heads = 0.0, 0.0, 0
+        while heads < H and t_tot < args.cpu_seconds:
+            f, dt = oracle_sample(qc[:, heads:heads + 1], kc[:, heads:heads + 1], vc[:, heads:heads + 1], posn, w,
+                                  1, N)
+            f_tot += f
+            t_tot += dt
+            heads += 1
+        cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"fp64 exact attention with RoPE on {heads} of 24 heads (all 16896 query rows each), "
+                         f"{t_tot:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "flux2k: Flux-like DiT joint attention at 2048 px, B=1 H=24 d=128 "
+                                   "N=512 text + 128x128 image = 16896, axes RoPE (16,56,56), theta 1e4, "
+                                   "Q/K 5% channels x8; gate on 16896x3072 bf16",
+                       "B": B, "H": H, "N": N, "d": d, "step": "rope(Q,K) + attn_bf16 + fbcache_gate",
+                       "l2": "inputs larger than L2 (Q+K+V+rotated Q,K = 519 MB per step > 126 MB)",
+                       "parallelism": f"independent problem per rank x{world}"},
+            "roofline": roofline,
+            "fp8": fp8,
+            "side_kernels": side,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": max(all_e2e) / ke},
+            "gpu_launches": args.steps * 4,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

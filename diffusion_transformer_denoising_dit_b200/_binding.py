@@ -1,0 +1,215 @@
+"""ctypes binding over libdit.so (argument marshalling only).
+
+Every operation runs in the library's sm_100a kernels on the caller's current
+CUDA stream; this module only checks tensor metadata, passes raw device
+pointers, element strides and sizes, and raises on a non-OK status.  There is
+no fallback: a missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdit.so")
+
+STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "DIT_ERR_ALIGNMENT",
+          4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT"}
+EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
+           "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
+           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate"]
+
+
+class DitError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+_i64x3 = ctypes.c_int64 * 3
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libdit.so; raises if it is absent (build it with build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m "
+                               "diffusion_transformer_denoising_dit_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.dit_status_string.restype = ctypes.c_char_p
+        L.dit_status_string.argtypes = [_i]
+        L.dit_read_error.restype = _i
+        L.dit_read_error.argtypes = [_vp]
+        L.dit_rope_tables.restype = _i
+        L.dit_rope_tables.argtypes = [_vp, _i, _i, _i, _i, ctypes.c_double, _vp, _vp, _vp]
+        L.rope_apply.restype = _i
+        L.rope_apply.argtypes = [_vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _vp, _vp, _i, _vp]
+        L.dit_attn_bf16_workspace_bytes.restype = _sz
+        L.dit_attn_bf16_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+        L.dit_attn_bf16.restype = _i
+        L.dit_attn_bf16.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _i64x3, _i64x3,
+                                    _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
+        L.dit_attn_fp8_workspace_bytes.restype = _sz
+        L.dit_attn_fp8_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+        L.dit_attn_fp8.restype = _i
+        L.dit_attn_fp8.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _i64x3, _i64x3,
+                                   _vp, _vp, ctypes.c_float, _i, _i, _i, _vp, _sz, _vp]
+        L.fbcache_gate_workspace_bytes.restype = _sz
+        L.fbcache_gate_workspace_bytes.argtypes = [ctypes.c_int64]
+        L.fbcache_gate.restype = _i
+        L.fbcache_gate.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise DitError(fn, code)
+
+
+def _stream(t: torch.Tensor):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _strides(t: torch.Tensor):
+    """{batch, head, token} element strides of a [B,H,N,d] tensor with a contiguous last dim."""
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    if t.stride(3) != 1:
+        raise ValueError("the channel (last) dimension must be contiguous")
+    return _i64x3(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+
+
+def read_error(stream=None) -> int:
+    """Synchronise the stream and return+clear the device error word (0 = none)."""
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return lib().dit_read_error(s)
+
+
+def rope_tables(pos: torch.Tensor, axes, theta: float = 10000.0):
+    """fp32 cos, sin tables [N, d/2] for int32 position ids pos [N, 3] (device)."""
+    _need_cuda(pos)
+    if pos.dtype != torch.int32 or pos.dim() != 2 or pos.shape[1] != 3:
+        raise ValueError("pos must be int32 [N, 3]")
+    pos = pos.contiguous()
+    N = pos.shape[0]
+    d = int(sum(axes))
+    c = torch.empty(N, d // 2, device=pos.device, dtype=torch.float32)
+    s = torch.empty_like(c)
+    _check("dit_rope_tables", lib().dit_rope_tables(pos.data_ptr(), N, int(axes[0]), int(axes[1]), int(axes[2]),
+                                                    float(theta), c.data_ptr(), s.data_ptr(), _stream(pos)))
+    return c, s
+
+
+def rope_apply(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, out_dtype=torch.bfloat16, out=None):
+    """Rotary embedding of x [B,H,N,d] (bf16) -> bf16 or fp32 (out may be x for in-place bf16)."""
+    _need_cuda(x, cos, sin)
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    B, H, N, d = x.shape
+    if out is None:
+        out = torch.empty(B, H, N, d, device=x.device, dtype=out_dtype)
+    dt = {torch.bfloat16: 0, torch.float32: 1}[out.dtype]
+    _check("rope_apply", lib().rope_apply(x.data_ptr(), out.data_ptr(), B, H, N, d, _strides(x), _strides(out),
+                                          cos.data_ptr(), sin.data_ptr(), dt, _stream(x)))
+    return out
+
+
+def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float | None = None,
+              out=None, workspace=None, q_block: int = 128, kv_block: int = 64, smooth_k: bool = True):
+    """Joint attention O [B,H,N,d] bf16 from bf16 q, k, v (+ optional rotary tables)."""
+    _need_cuda(q, k, v, cos, sin)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be bf16")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same [B, H, N, d] shape")
+    B, H, N, d = q.shape
+    if out is None:
+        out = torch.empty(B, H, N, d, device=q.device, dtype=torch.bfloat16)
+    sc = 0.0 if scale is None else float(scale)
+    L = lib()
+    if precision == "bf16":
+        need = L.dit_attn_bf16_workspace_bytes(B, H, N, d, int(cos is not None))
+    elif precision == "fp8":
+        need = L.dit_attn_fp8_workspace_bytes(B, H, N, d, q_block, kv_block)
+    else:
+        raise ValueError("precision must be 'bf16' or 'fp8'")
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    wp = _ptr(workspace) if need else None
+    wb = need if need else 0
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
+            _strides(q), _strides(k), _strides(v), _strides(out), _ptr(cos), _ptr(sin), sc)
+    if precision == "bf16":
+        _check("dit_attn_bf16", L.dit_attn_bf16(*args, wp, wb, _stream(q)))
+    else:
+        _check("dit_attn_fp8", L.dit_attn_fp8(*args, q_block, kv_block, int(smooth_k), wp, wb, _stream(q)))
+    return out
+
+
+def attention_workspace(B, H, N, d, precision="bf16", rope=True, q_block=128, kv_block=64, device="cuda"):
+    """Pre-allocated workspace for repeated attention calls of one shape."""
+    L = lib()
+    need = (L.dit_attn_bf16_workspace_bytes(B, H, N, d, int(rope)) if precision == "bf16"
+            else L.dit_attn_fp8_workspace_bytes(B, H, N, d, q_block, kv_block))
+    return torch.empty(max(need, 1), device=device, dtype=torch.uint8)
+
+
+def fbcache_gate(r_cur, r_prev, threshold: float, rel_out=None, skip_out=None, workspace=None):
+    """(rel fp32 [1], skip int32 [1]) device tensors for two bf16 residuals of equal size."""
+    _need_cuda(r_cur, r_prev)
+    if r_cur.dtype != torch.bfloat16 or r_prev.dtype != torch.bfloat16:
+        raise ValueError("residuals must be bf16")
+    if r_cur.numel() != r_prev.numel() or not r_cur.is_contiguous() or not r_prev.is_contiguous():
+        raise ValueError("residuals must be contiguous and of equal size")
+    n = r_cur.numel()
+    L = lib()
+    need = L.fbcache_gate_workspace_bytes(n)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, device=r_cur.device, dtype=torch.uint8)
+    if rel_out is None:
+        rel_out = torch.empty(1, device=r_cur.device, dtype=torch.float32)
+    if skip_out is None:
+        skip_out = torch.empty(1, device=r_cur.device, dtype=torch.int32)
+    _check("fbcache_gate", L.fbcache_gate(r_cur.data_ptr(), r_prev.data_ptr(), n, float(threshold),
+                                          rel_out.data_ptr(), skip_out.data_ptr(), workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(), _stream(r_cur)))
+    return rel_out, skip_out
+
+
+class FBCacheGate:
+    """First-Block-Cache decision with its buffers allocated once.
+
+    gate(r_cur, r_prev) enqueues the kernels and returns the device int32
+    skip flag; ``.rel`` holds the relative L1 change.  Reading the flag on the
+    host (``bool(flag.item())``) is the one device-to-host crossing per step.
+    """
+
+    def __init__(self, threshold: float, numel: int, device="cuda"):
+        self.threshold = float(threshold)
+        self.rel = torch.empty(1, device=device, dtype=torch.float32)
+        self.skip = torch.empty(1, device=device, dtype=torch.int32)
+        self.workspace = torch.empty(lib().fbcache_gate_workspace_bytes(numel), device=device, dtype=torch.uint8)
+
+    def __call__(self, r_cur, r_prev):
+        fbcache_gate(r_cur, r_prev, self.threshold, self.rel, self.skip, self.workspace)
+        return self.skip

@@ -1,0 +1,74 @@
+// Internal launcher interface between the C ABI (capi.cu) and the kernel
+// translation units.  Not part of the public header.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace dit {
+
+// Error codes written to the device error word (match dit_status).
+constexpr int kErrTimeout = 6;
+
+// Gate: number of pass-1 CTAs for n elements, and its workspace (2 doubles per CTA).
+int gate_num_ctas(int64_t n);
+
+cudaError_t launch_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, double theta, float* cos_out,
+                               float* sin_out, cudaStream_t stream);
+
+// One strided [B,H,N,d] rotary job.
+struct RopeJob {
+  const void* x;
+  void* y;
+  int64_t sx[3];
+  int64_t sy[3];
+};
+
+// Applies rotary embedding to njobs (1 or 2) tensors of the same shape in one launch.
+cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int N, int d, const float* cos_tab,
+                              const float* sin_tab, int out_fp32, cudaStream_t stream);
+
+cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold, float* rel_out, int32_t* skip_out,
+                        double* partials, cudaStream_t stream);
+
+// Output description shared by the attention kernels.
+struct AttnOut {
+  void* o;          // bf16 [B,H,N,d]
+  int64_t so[3];    // element strides {batch, head, token}
+  int N;
+  float scale_log2;  // softmax scale * log2(e)
+  int* err;          // device error word
+};
+
+cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
+                             int B, int H, int d, cudaStream_t stream);
+
+// FP8 prologue: K channel means (fp32 [B*H][d]) of the rotated K.
+struct Fp8Prep {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t sq[3], sk[3], sv[3];
+  const float* cos_tab;  // may be null (no rotary)
+  const float* sin_tab;
+  int B, H, N, d;
+  int q_block, kv_block;
+  int smooth_k;
+  // workspace carve-out
+  uint8_t* q8;      // e4m3 [B,H,N,d]
+  uint8_t* k8;      // e4m3 [B,H,N,d]
+  uint8_t* v8;      // e4m3 [B,H,N,d]
+  float* q_scale;   // [B*H][ceil(N/q_block)]
+  float* k_scale;   // [B*H][ceil(N/kv_block)]
+  float* v_scale;   // [B*H][ceil(N/kv_block)]
+  float* k_mean;    // [B*H][d]
+  float* v_scale_max;  // [B*H]
+};
+
+cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream);
+
+cudaError_t launch_attn_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
+                            const Fp8Prep& p, cudaStream_t stream);
+
+}  // namespace dit

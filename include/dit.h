@@ -1,0 +1,158 @@
+/*
+ * dit.h -- C ABI of the B200 (sm_100a) DiT joint-attention hot path.
+ *
+ * The operations, and the pages they are read from:
+ *
+ *   dit_attn_bf16    joint image+text multi-head self-attention with rotary
+ *                    embedding on Q and K, BF16 operands, fp32 accumulation.
+ *                    "FLUX 3 Image Klein / TensorRT-LLM VisualGen", section on
+ *                    why the differences arise: the DiT's VANILLA BF16
+ *                    attention takes about 60 % of its GPU kernel time.
+ *   dit_attn_fp8     the same attention with e4m3 Q/K/V quantised in
+ *                    per-token blocks, K mean-smoothed before quantisation.
+ *                    Same page (cuDNN FP8 attention against VANILLA BF16) and
+ *                    "vflash / Optimization ledger", table "Accepted or
+ *                    exposed" (SageAttention2, a quantised attention).
+ *   dit_rope_tables  cos/sin tables of the multi-axis rotary embedding.
+ *   rope_apply       rotary embedding applied to a [B,H,N,d] tensor.
+ *                    "vflash / Optimization ledger", row "strict Triton RoPE".
+ *   fbcache_gate     First-Block-Cache decision: relative L1 change of the
+ *                    first block's residual between consecutive denoising
+ *                    steps, compared with a threshold.  unsloth studio commit
+ *                    "core/inference/diffusion.py", paragraph "Add opt-in step
+ *                    caching (First-Block-Cache)".
+ *
+ * Definitions (the pages name these operations without formulas; the plain
+ * textbook readings are used):
+ *
+ *   attention   O[b,h,i,:] = sum_j softmax_j(s_ij) V[b,h,j,:],
+ *               s_ij = scale * <R_i Q[b,h,i,:], R_j K[b,h,j,:]>, every j in
+ *               0..N-1 (bidirectional, no mask), scale <= 0 means 1/sqrt(d).
+ *   rotary      head dim split into axis slices (d0,d1,d2), all even; pair p
+ *               of axis a = channels (off_a+2p, off_a+2p+1), rotated by
+ *               pos[a]*theta^(-2p/d_a):  y0 = x0 c - x1 s,  y1 = x0 s + x1 c.
+ *               Tables hold c and s as fp32 [N][d/2] (pair index global).
+ *   gate        rel = sum|r_cur - r_prev| / sum|r_prev| (0 if both sums are
+ *               0, +inf if only the denominator is), skip = rel < threshold.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller (e.g. by
+ *     PyTorch).  The library never allocates, frees or synchronises, except
+ *     dit_read_error which synchronises the given stream.
+ *   - Tensors [B,H,N,d] are described by element strides {batch, head,
+ *     token}; the channel dimension is contiguous.  Strides and base pointers
+ *     must be 16-byte aligned (a TMA requirement): bf16 strides multiple of 8.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - A non-DIT_OK return means nothing was enqueued.  Failures inside a
+ *     kernel (a bounded wait that ran out) are recorded in a device error
+ *     word that dit_read_error returns and clears.
+ *   - There is no CPU fallback: every call runs the sm_100a kernels, and
+ *     returns DIT_ERR_UNSUPPORTED on any other device.
+ */
+#ifndef DIT_H_
+#define DIT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DIT_API __attribute__((visibility("default")))
+#else
+#define DIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dit_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  DIT_OK = 0,
+  DIT_ERR_INVALID_ARG = 1,  /* null pointer, bad size or shape */
+  DIT_ERR_UNSUPPORTED = 2,  /* d not supported, device not sm_100 */
+  DIT_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
+  DIT_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+  DIT_ERR_LAUNCH = 5,       /* CUDA error while enqueueing */
+  DIT_ERR_TIMEOUT = 6       /* (device error word) a bounded wait ran out */
+} dit_status;
+
+/* Human-readable name of a status code (static string). */
+DIT_API const char* dit_status_string(dit_status s);
+
+/* Synchronises `stream`, then returns and clears the device error word of the
+ * current device (DIT_OK if no kernel recorded a failure). */
+DIT_API dit_status dit_read_error(dit_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Rotary embedding                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Builds cos/sin tables, fp32 [N][d/2] each, d = d0+d1+d2, from int32
+ * position ids pos[N][3] (device).  Angles are formed and evaluated in fp64
+ * and rounded once to fp32.  d0,d1,d2 even and >= 0, d <= 256, N >= 1. */
+DIT_API dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, double theta, float* cos_out,
+                           float* sin_out, dit_stream_t stream);
+
+/* y = rotary(x) for x, y [B,H,N,d] with element strides sx/sy {batch, head,
+ * token}; y may alias x exactly (in place).  dtype: 0 = bf16 in and out,
+ * 1 = bf16 in, fp32 out.  Math in fp32, output rounded once (RNE).
+ * d in {64, 128}; tables as built by dit_rope_tables. */
+DIT_API dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d, const int64_t sx[3], const int64_t sy[3],
+                      const float* cos_tab, const float* sin_tab, int dtype, dit_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Attention                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace needed by dit_attn_bf16 (0 when has_rope == 0).  With rotary
+ * tables the rotated Q and K are staged there as contiguous bf16 [B,H,N,d]. */
+DIT_API size_t dit_attn_bf16_workspace_bytes(int B, int H, int N, int d, int has_rope);
+
+/* O = attention(Q, K, V) in BF16 with fp32 accumulation and softmax.
+ * q, k, v: bf16 [B,H,N,d] inputs; o: bf16 [B,H,N,d] output (must not alias
+ * q, k or v).  rope_cos/rope_sin: tables [N][d/2] or both NULL (no rotary).
+ * softmax_scale <= 0 selects 1/sqrt(d).  d in {64, 128}; N >= 1.
+ * workspace: device buffer of at least dit_attn_bf16_workspace_bytes, 256-byte
+ * aligned (may be NULL when that size is 0). */
+DIT_API dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                         const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
+                         size_t workspace_bytes, dit_stream_t stream);
+
+/* Workspace needed by dit_attn_fp8: e4m3 copies of rotated Q, smoothed K
+ * and V, their per-block fp32 scales and the fp32 K channel means. */
+DIT_API size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_block, int kv_block);
+
+/* O = attention in FP8: Q, K, V rotated (Q, K), K smoothed (smooth_k != 0:
+ * per-(b,h) channel mean over all N tokens subtracted after rotation), then
+ * quantised to e4m3 (RNE, saturating) with one fp32 scale amax/448 per block
+ * of q_block (Q) or kv_block (K, V) tokens.  Scores accumulate in fp32; P is
+ * e4m3 with the V block scale folded in; the row sum uses the fp32 P.
+ * Supported: d = 128, q_block = 128, kv_block = 64.  Arguments otherwise as
+ * dit_attn_bf16. */
+DIT_API dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                        const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                        const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
+                        int smooth_k, void* workspace, size_t workspace_bytes, dit_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* First-Block-Cache gate                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace needed by fbcache_gate for n elements (per-CTA partial sums). */
+DIT_API size_t fbcache_gate_workspace_bytes(int64_t n);
+
+/* rel_out[0] = sum|r_cur - r_prev| / sum|r_prev| over n contiguous bf16
+ * elements (fp32 per-thread partials, fp64 combine in a fixed order, so the
+ * result is deterministic); skip_out[0] = (rel < threshold).  rel_out and
+ * skip_out are device pointers; read skip_out on the host to branch.
+ * n >= 1; r_cur, r_prev 16-byte aligned. */
+DIT_API dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float threshold, float* rel_out,
+                        int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_H_ */

@@ -1,0 +1,92 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/dit.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from diffusion_transformer_denoising_dit_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dit.h")
+
+pytestmark = pytest.mark.skipif(not os.path.exists(B.LIB_PATH), reason="libdit.so not built (run build())")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"DIT_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = B.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = B.lib()
+    for code, name in B.STATUS.items():
+        assert L.dit_status_string(code).decode() == name
+
+
+S = B._i64x3
+A16 = 1 << 20          # a fake 16-byte aligned device address (never dereferenced)
+
+
+def _attn(L, q=A16, k=A16, v=A16, o=A16, Bn=1, H=1, N=16, d=64, s=(1024, 1024, 64), cos=None, sin=None,
+          scale=0.0, ws=None, wsb=0):
+    st = S(*s)
+    return L.dit_attn_bf16(q, k, v, o, Bn, H, N, d, st, st, st, st, cos, sin, scale, ws, wsb, None)
+
+
+def test_attention_argument_validation():
+    L = B.lib()
+    assert _attn(L, q=None) == 1                      # null pointer
+    assert _attn(L, N=0) == 1                         # empty sequence
+    assert _attn(L, d=96) == 2                        # unsupported head dim
+    assert _attn(L, q=A16 + 2) == 3                   # misaligned base
+    assert _attn(L, s=(1024, 1024, 60)) == 3          # token stride not 16-byte aligned
+    assert _attn(L, cos=A16) == 3                     # only one of the two tables
+    assert _attn(L, cos=A16, sin=A16) == 4            # RoPE needs a workspace
+    need = L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 1)
+    assert need == 2 * (2 * 16 * 64)                 # rotated Q and K, bf16, 256-byte aligned
+    assert _attn(L, cos=A16, sin=A16, ws=A16, wsb=need - 1) == 4
+    assert L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 0) == 0
+
+
+def test_fp8_argument_validation():
+    L = B.lib()
+    st = S(1024 * 128, 1024 * 128, 128)
+    args = (A16, A16, A16, A16, 1, 1, 1024, 128, st, st, st, st, None, None, 0.0)
+    assert L.dit_attn_fp8(*args, 64, 64, 1, A16, 1 << 30, None) == 2      # q_block != 128
+    assert L.dit_attn_fp8(*args, 128, 64, 1, None, 0, None) == 4          # no workspace
+    small = L.dit_attn_fp8_workspace_bytes(1, 1, 1024, 128, 128, 64) - 1
+    assert L.dit_attn_fp8(*args, 128, 64, 1, A16, small, None) == 4
+
+
+def test_gate_and_rope_validation():
+    L = B.lib()
+    assert L.fbcache_gate(A16, A16, 0, 0.1, A16, A16, A16, 1 << 20, None) == 1      # n = 0
+    assert L.fbcache_gate(A16 + 4, A16, 100, 0.1, A16, A16, A16, 1 << 20, None) == 3
+    assert L.fbcache_gate(A16, A16, 100, 0.1, A16, A16, A16, 1, None) == 4           # workspace too small
+    assert L.fbcache_gate_workspace_bytes(100) == 16
+    assert L.dit_rope_tables(A16, 10, 16, 24, 25, 1e4, A16, A16, None) == 1          # odd axis width
+    assert L.dit_rope_tables(A16, 10, 16, 24, 24, -1.0, A16, A16, None) == 1         # bad theta
+    st = S(4096, 4096, 64)
+    assert L.rope_apply(A16, A16, 1, 1, 64, 64, st, st, A16, A16, 1, None) == 1      # fp32 out in place
+    assert L.rope_apply(A16, A16, 1, 1, 64, 48, st, st, A16, A16, 0, None) == 2      # d = 48
+
+
+def test_no_gpu_means_unsupported_not_fallback():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    L = B.lib()
+    assert _attn(L) == 2
+    assert L.fbcache_gate(A16, A16, 100, 0.1, A16, A16, A16, 1 << 20, None) == 2

@@ -1,0 +1,130 @@
+"""GPU parity of dit_attn_bf16 against the fp64 oracle.
+
+Bar (BF16): max |O - O_ref| <= 2e-2 and cosine >= 0.9999 against exact fp64
+attention on the same bf16 inputs.  Small workloads are compared element by
+element over the whole output; the 2048-px workload, in the launch
+configuration the benchmark times, on sampled query rows of every head
+(including the first and last tile).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import cuda_ok
+from oracle import attention as A
+from diffusion_transformer_denoising_dit_b200 import synth
+import diffusion_transformer_denoising_dit_b200 as dit
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA GPU")]
+DEV = "cuda"
+MAX_ABS = 2e-2
+MIN_COS = 0.9999
+
+
+def _cos(a, b):
+    return float((a * b).sum() / math.sqrt((a * a).sum() * (b * b).sum()))
+
+
+def _check(o, ref, max_abs=MAX_ABS, min_cos=MIN_COS):
+    o = o.cpu().double().numpy() if isinstance(o, torch.Tensor) else o
+    err = np.abs(o - ref).max()
+    cs = _cos(o, ref)
+    assert err <= max_abs and cs >= min_cos, (err, cs)
+    return err, cs
+
+
+def _run(w, N=None, B=None, rope=True, rows=None, seed=None, layout="bhnd"):
+    q, k, v = synth.qkv(w, device=DEV, N=N, B=B, seed=seed)
+    Nn = q.shape[2]
+    if layout == "bnhd":
+        q, k, v = (t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3) for t in (q, k, v))
+    pos = None
+    cos = sin = None
+    if rope and w.rope:
+        pos = synth.positions(w.T, w.G) if N is None else _positions_for(w, Nn)
+        cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+        pos = pos.numpy()
+    o = dit.attention(q, k, v, cos, sin)
+    torch.cuda.synchronize()
+    assert dit.read_error() == 0
+    ref = A.attention(q.cpu(), k.cpu(), v.cpu(), pos=pos, axes=w.axes, theta=w.theta, rows=rows)
+    if rows is not None:
+        o = o[:, :, rows]
+    return o, ref
+
+
+def _positions_for(w, N):
+    """Text then a row-major image grid truncated to N tokens (ragged sequences)."""
+    full = synth.positions(w.T, int(math.isqrt(max(N - w.T, 1))) + 1)
+    return full[:N].contiguous()
+
+
+def test_tiny_full_output():
+    _check(*_run(synth.WORKLOADS["tiny"]))
+
+
+def test_tiny_without_rope():
+    _check(*_run(synth.WORKLOADS["tiny"], rope=False))
+
+
+def test_sdxl_full_output():
+    _check(*_run(synth.WORKLOADS["sdxl"]))
+
+
+@pytest.mark.parametrize("N", [1, 2, 100, 127, 128, 129, 255, 300, 1000])
+def test_ragged_lengths_d64(N):
+    _check(*_run(synth.WORKLOADS["tiny"], N=N, seed=N))
+
+
+@pytest.mark.parametrize("N", [1, 129, 513, 777])
+def test_ragged_lengths_d128(N):
+    w = synth.WORKLOADS["flux1k"]
+    import dataclasses
+    w = dataclasses.replace(w, H=3, T=min(N, 64))
+    _check(*_run(w, N=N, seed=N))
+
+
+def test_flux1k_full_output_two_heads_and_strided_layout():
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2)
+    _check(*_run(w, layout="bnhd"))
+
+
+def test_batch_and_heads_grid():
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["tiny"], H=5)
+    _check(*_run(w, B=3, N=200, seed=5))
+
+
+def test_flux1k_all_heads_sampled_rows():
+    w = synth.WORKLOADS["flux1k"]
+    rows = np.unique(np.concatenate([np.arange(0, 128), np.arange(4480, 4608),
+                                     np.random.default_rng(1).integers(0, 4608, 256)]))
+    _check(*_run(w, rows=rows))
+
+
+def test_flux2k_bench_configuration_sampled_rows():
+    """The benchmark's workload (B=1, H=24, N=16896, d=128, RoPE) at full size."""
+    w = synth.WORKLOADS["flux2k"]
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(16896 - 64, 16896),
+                                     np.random.default_rng(2).integers(0, 16896, 128)]))
+    _check(*_run(w, rows=rows))
+
+
+def test_explicit_scale_and_zero_q():
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w, device=DEV)
+    o = dit.attention(torch.zeros_like(q), k, v)
+    ref_mean = v.double().mean(dim=2, keepdim=True).expand_as(v)
+    assert (o.double() - ref_mean).abs().max().item() <= 1e-2
+    o2 = dit.attention(q, k, v, scale=0.05)
+    ref = A.attention(q.cpu(), k.cpu(), v.cpu(), scale=0.05)
+    _check(o2, ref)
+
+
+def test_repeat_calls_are_deterministic():
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w, device=DEV)
+    assert torch.equal(dit.attention(q, k, v), dit.attention(q, k, v))
