@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     attention,
     attention_workspace,
     fbcache_gate,
+    fp8_workspace_views,
     lib,
     read_error,
     rope_apply,

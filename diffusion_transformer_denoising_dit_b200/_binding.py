@@ -174,6 +174,34 @@ def attention_workspace(B, H, N, d, precision="bf16", rope=True, q_block=128, kv
     return torch.empty(max(need, 1), device=device, dtype=torch.uint8)
 
 
+def _a256(x: int) -> int:
+    return (x + 255) // 256 * 256
+
+
+def fp8_workspace_views(ws: torch.Tensor, B: int, H: int, N: int, d: int = 128, q_block: int = 128,
+                        kv_block: int = 64):
+    """Views into a dit_attn_fp8 workspace (the layout written by the FP8 prologue):
+    q8, k8, v8 (uint8 e4m3 codes [B,H,N,d]), q_scale, k_scale, v_scale, k_mean, v_scale_max."""
+    bh = B * H
+    el = bh * N * d
+    nq, nk = -(-N // q_block), -(-N // kv_block)
+    off = 0
+    out = {}
+    for name in ("q8", "k8", "v8"):
+        out[name] = ws[off:off + el].view(B, H, N, d)
+        off += _a256(el)
+    for name, n in (("q_scale", bh * nq), ("k_scale", bh * nk), ("v_scale", bh * nk), ("k_mean", bh * d),
+                    ("v_scale_max", bh)):
+        out[name] = ws[off:off + 4 * n].view(torch.float32)
+        off += _a256(4 * n)
+    out["q_scale"] = out["q_scale"].view(B, H, nq)
+    out["k_scale"] = out["k_scale"].view(B, H, nk)
+    out["v_scale"] = out["v_scale"].view(B, H, nk)
+    out["k_mean"] = out["k_mean"].view(B, H, d)
+    out["v_scale_max"] = out["v_scale_max"].view(B, H)
+    return out
+
+
 def fbcache_gate(r_cur, r_prev, threshold: float, rel_out=None, skip_out=None, workspace=None):
     """(rel fp32 [1], skip int32 [1]) device tensors for two bf16 residuals of equal size."""
     _need_cuda(r_cur, r_prev)

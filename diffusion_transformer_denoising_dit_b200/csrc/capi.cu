@@ -223,7 +223,7 @@ size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_block, int
   const size_t el = bh * N * d;
   const size_t nq = (N + q_block - 1) / q_block, nk = (N + kv_block - 1) / kv_block;
   return 3 * align256(el) + align256(bh * nq * 4) + 2 * align256(bh * nk * 4) + align256(bh * d * 4) +
-         align256(bh * 4);
+         align256(bh * 4) + align256(bh * dit::kFp8MeanChunks * d * 4);
 }
 
 dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
@@ -262,7 +262,8 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   p.k_scale = reinterpret_cast<float*>(w); w += align256(bh * nk * 4);
   p.v_scale = reinterpret_cast<float*>(w); w += align256(bh * nk * 4);
   p.k_mean = reinterpret_cast<float*>(w); w += align256(bh * d * 4);
-  p.v_scale_max = reinterpret_cast<float*>(w);
+  p.v_scale_max = reinterpret_cast<float*>(w); w += align256(bh * 4);
+  p.k_partial = reinterpret_cast<float*>(w);
 
   if (dit::launch_fp8_prologue(p, st) != cudaSuccess) return DIT_ERR_LAUNCH;
   const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};

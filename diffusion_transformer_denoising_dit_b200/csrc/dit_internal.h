@@ -64,7 +64,10 @@ struct Fp8Prep {
   float* v_scale;   // [B*H][ceil(N/kv_block)]
   float* k_mean;    // [B*H][d]
   float* v_scale_max;  // [B*H]
+  float* k_partial;    // [B*H][kFp8MeanChunks][128] K-mean partial sums
 };
+
+constexpr int kFp8MeanChunks = 16;
 
 cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream);
 

@@ -1,0 +1,231 @@
+// FP8 prologue: rotary embedding, K mean-smoothing and per-block e4m3
+// quantisation of Q, K and V, ahead of the FP8 attention kernel.
+//
+// Sources: "FLUX 3 Image Klein / TensorRT-LLM VisualGen" (cuDNN FP8 attention
+// against VANILLA BF16) and "vflash / Optimization ledger", table "Accepted or
+// exposed" (SageAttention2: quantised attention).  Neither page fixes the
+// scheme; the readings: e4m3 (RNE, saturating), one fp32 scale amax/448 per
+// block of 128 (Q) or 64 (K, V) tokens of one (batch, head), K minus its
+// channel mean over all N tokens after rotation (which leaves softmax
+// unchanged in exact arithmetic).
+//
+// Pass 1 (kmean_partial): per (b,h) and token chunk, fp32 channel sums of the
+//   rotated K; also clears the per-(b,h) V scale maximum.
+// Pass 2 (quantize): one CTA per (b,h, 128-token block): rotate Q and K in
+//   fp32, subtract the K mean (partials combined in a fixed order), block
+//   amax, scale and cast to e4m3; write the scales.  Streams 6 B/element in
+//   (bf16 Q, K, V) and 3 B/element out; HBM-bound.
+#include <cuda_bf16.h>
+
+#include "dit_device.cuh"
+
+namespace dit {
+namespace {
+
+constexpr int kChunks = kFp8MeanChunks;  // token chunks of the K-mean pass per (b,h)
+constexpr int kThreads = 256;  // 16 channel chunks (8 channels each) x 16 token lanes
+
+__device__ __forceinline__ void load_rotate8(const __nv_bfloat16* __restrict__ src, const float* __restrict__ cos_tab,
+                                             const float* __restrict__ sin_tab, int n, int cc, int half_d,
+                                             float (&y)[8]) {
+  const uint4 xv = *reinterpret_cast<const uint4*>(src);
+  const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
+  if (cos_tab) {
+    const float4 cv = *reinterpret_cast<const float4*>(cos_tab + static_cast<int64_t>(n) * half_d + cc * 4);
+    const float4 sv = *reinterpret_cast<const float4*>(sin_tab + static_cast<int64_t>(n) * half_d + cc * 4);
+    const float c4[4] = {cv.x, cv.y, cv.z, cv.w};
+    const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(xp[i]);
+      y[2 * i] = x.x * c4[i] - x.y * s4[i];
+      y[2 * i + 1] = x.x * s4[i] + x.y * c4[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(xp[i]);
+      y[2 * i] = x.x;
+      y[2 * i + 1] = x.y;
+    }
+  }
+}
+
+// Two floats -> two e4m3 bytes (round to nearest even, saturating); lo in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+__global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __restrict__ partial) {
+  const int bh = blockIdx.y;
+  const int chunk = blockIdx.x;
+  if (chunk == 0 && threadIdx.x == 0) p.v_scale_max[bh] = 0.f;
+  const int b = bh / p.H, h = bh % p.H;
+  const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
+  const int per = (p.N + kChunks - 1) / kChunks;
+  const int n0 = chunk * per, n1 = min(p.N, n0 + per);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (p.smooth_k) {
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
+    for (int n = n0 + tl; n < n1; n += 16) {
+      float y[8];
+      load_rotate8(kb + static_cast<int64_t>(n) * p.sk[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, p.d / 2, y);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += y[i];
+    }
+  }
+  __shared__ float red[16][128 + 4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[tl][cc * 8 + i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) s += red[r][threadIdx.x];
+    partial[(static_cast<int64_t>(bh) * kChunks + chunk) * 128 + threadIdx.x] = s;
+  }
+}
+
+// Quantises one 128-token block of one tensor held as 8 chunks per thread:
+// thread t owns channel chunk (t % 16) of tokens t/16 + 16 i, i = 0..7.  With
+// two_blocks the first four tokens of a thread lie in the first 64-token block.
+__device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks, int n_base, int N,
+                                              uint8_t* __restrict__ dst, int cc, int tl, float* red, float* sc_out0,
+                                              float* sc_out1, float* vmax) {
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (i < 4 || !two_blocks)
+        a0 = fmaxf(a0, fabsf(x[i][e]));
+      else
+        a1 = fmaxf(a1, fabsf(x[i][e]));
+    }
+  a0 = block_max(a0, red);
+  if (two_blocks) a1 = block_max(a1, red + 8);
+  const float s0 = a0 > 0.f ? a0 / 448.f : 1.f;
+  const float s1 = a1 > 0.f ? a1 / 448.f : 1.f;
+  const float inv0 = a0 > 0.f ? 448.f / a0 : 1.f;
+  const float inv1 = a1 > 0.f ? 448.f / a1 : 1.f;
+  if (threadIdx.x == 0) {
+    *sc_out0 = s0;
+    if (two_blocks) *sc_out1 = s1;
+    if (vmax) {
+      atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s0));
+      if (two_blocks) atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s1));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = n_base + tl + 16 * i;
+    if (n >= N) continue;
+    const float inv = (i < 4 || !two_blocks) ? inv0 : inv1;
+    uint2 w;
+    w.x = cvt_e4m3x2(x[i][0] * inv, x[i][1] * inv) | (cvt_e4m3x2(x[i][2] * inv, x[i][3] * inv) << 16);
+    w.y = cvt_e4m3x2(x[i][4] * inv, x[i][5] * inv) | (cvt_e4m3x2(x[i][6] * inv, x[i][7] * inv) << 16);
+    *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(n) * 128 + cc * 8) = w;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) quantize_qkv(Fp8Prep p, const float* __restrict__ partial) {
+  const int blk = blockIdx.x;  // 128-token block
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
+  const int n_base = blk * 128;
+  const int nq = (p.N + 127) / 128, nk = (p.N + 63) / 64;
+  __shared__ float mean[128];
+  __shared__ float red[16];
+  __shared__ float unused_scale;  // sink for the second scale of a block past the sequence end
+  if (threadIdx.x < 128) {
+    float s = 0.f;
+    if (p.smooth_k)
+      for (int c = 0; c < kChunks; ++c) s += partial[(static_cast<int64_t>(bh) * kChunks + c) * 128 + threadIdx.x];
+    const float m = s / static_cast<float>(p.N);
+    mean[threadIdx.x] = m;
+    if (blk == 0) p.k_mean[bh * 128 + threadIdx.x] = m;
+  }
+  __syncthreads();
+  const int64_t out_off = static_cast<int64_t>(bh) * p.N * 128;
+  float x[8][8];
+  // ---- Q: one 128-token block
+  {
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.q) + b * p.sq[0] + h * p.sq[1];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int n = n_base + tl + 16 * i;
+      if (n < p.N)
+        load_rotate8(src + static_cast<int64_t>(n) * p.sq[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, 64, x[i]);
+      else
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+    }
+    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr);
+  }
+  // ---- K: two 64-token blocks, smoothed
+  {
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int n = n_base + tl + 16 * i;
+      if (n < p.N) {
+        load_rotate8(src + static_cast<int64_t>(n) * p.sk[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, 64, x[i]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] -= mean[cc * 8 + e];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+      }
+    }
+    float* s1 = (2 * blk + 1 < nk) ? p.k_scale + bh * nk + 2 * blk + 1 : &unused_scale;
+    quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr);
+  }
+  // ---- V: two 64-token blocks, no rotation
+  {
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.v) + b * p.sv[0] + h * p.sv[1];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int n = n_base + tl + 16 * i;
+      if (n < p.N)
+        load_rotate8(src + static_cast<int64_t>(n) * p.sv[2] + cc * 8, nullptr, nullptr, n, cc, 64, x[i]);
+      else
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+    }
+    const bool has2 = 2 * blk + 1 < nk;
+    float* s1 = has2 ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
+    quantize_tile(x, true, n_base, p.N, p.v8 + out_off, cc, tl, red, p.v_scale + bh * nk + 2 * blk, s1,
+                  p.v_scale_max + bh);
+  }
+  (void)nq;
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
+  float* partial = p.k_partial;
+  dim3 g1(kChunks, p.B * p.H);
+  kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 g2((p.N + 127) / 128, p.B * p.H);
+  quantize_qkv<<<g2, kThreads, 0, stream>>>(p, partial);
+  return cudaGetLastError();
+}
+
+}  // namespace dit

@@ -22,6 +22,22 @@ import numpy as np
 from . import rope as _rope
 
 
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (8 significant bits), ties to even.
+
+    bfloat16 keeps float32's exponent range and 7 stored mantissa bits; the
+    values met here are normal, so the spacing in binade [2^e, 2^(e+1)) is
+    2^(e-7).  Zero stays zero.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.abs(x)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    e = np.maximum(e, -126.0)
+    q = np.exp2(e - 7)
+    return np.copysign(np.round(ax / q) * q, x)
+
+
 def _f64(t) -> np.ndarray:
     """Exact fp64 copy of a tensor/array (bf16 values upcast exactly)."""
     try:
@@ -42,14 +58,23 @@ def rotate(x, pos, axes, theta):
 
 
 def attention(q, k, v, scale=None, pos=None, axes=None, theta=10000.0,
-              rows=None, chunk=1024) -> np.ndarray:
+              rows=None, chunk=1024, operands=None) -> np.ndarray:
     """fp64 O for q, k, v of shape [B, H, N, d].
 
     rows: optional 1-D index array of query rows to evaluate (same for every
     (b, h)); the result then has shape [B, H, len(rows), d].
+    operands: None keeps the rotated Q and K exact; "bf16" rounds them once to
+    bfloat16, the reading of the BF16 variant (its tensor-core operands are the
+    rotated Q and K as bf16 tensors, as when a RoPE kernel writes bf16 that a
+    BF16 attention kernel reads).  Without rotation the inputs are bf16 already.
     """
     q = rotate(q, pos, axes, theta)
     k = rotate(k, pos, axes, theta)
+    if operands == "bf16":
+        q = round_bf16(q)
+        k = round_bf16(k)
+    elif operands is not None:
+        raise ValueError("operands must be None or 'bf16'")
     v = _f64(v)
     B, H, N, d = q.shape
     sigma = 1.0 / math.sqrt(d) if scale is None or scale <= 0 else float(scale)

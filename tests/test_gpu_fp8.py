@@ -1,0 +1,121 @@
+"""GPU checks of the FP8 path: the prologue against the oracle's quantiser, and
+dit_attn_fp8 against the simulated-FP8 diagnostic and the exact oracle.
+
+Bars: on N(0,1) inputs cosine >= 0.995 against exact fp64 attention (the
+target).  On the workloads with x8 outlier channels the e4m3 Q.K^T floor of
+any such scheme sits near 0.98 (oracle diagnostic), so there the kernel must
+match the simulated-FP8 oracle (cosine >= 0.999) and come within 0.005 of
+that floor against the exact result.
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import cuda_ok
+from oracle import attention as A
+from oracle import fp8 as F
+from oracle import rope as R
+from diffusion_transformer_denoising_dit_b200 import synth
+import diffusion_transformer_denoising_dit_b200 as dit
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA GPU")]
+DEV = "cuda"
+
+
+def _cos(a, b):
+    return float((a * b).sum() / math.sqrt((a * a).sum() * (b * b).sum()))
+
+
+def _inputs(w, N=None, seed=None):
+    q, k, v = synth.qkv(w, device=DEV, N=N, seed=seed)
+    Nn = q.shape[2]
+    pos = synth.positions(w.T, w.G) if N is None else synth.positions(w.T, int(math.isqrt(max(Nn - w.T, 1))) + 1)[:Nn]
+    cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    return q, k, v, pos.numpy(), cos, sin
+
+
+def _run(w, N=None, seed=None, rows=None, smooth=True):
+    q, k, v, pos, cos, sin = _inputs(w, N, seed)
+    ws = dit.attention_workspace(*q.shape, precision="fp8", device=DEV)
+    o = dit.attention(q, k, v, cos, sin, precision="fp8", workspace=ws, smooth_k=smooth)
+    assert dit.read_error() == 0
+    args = dict(pos=pos, axes=w.axes, theta=w.theta, rows=rows)
+    exact = A.attention(q.cpu(), k.cpu(), v.cpu(), **args)
+    sim = F.simulated_attention(q.cpu(), k.cpu(), v.cpu(), smooth=smooth, **args)
+    o = o.cpu().double().numpy()
+    if rows is not None:
+        o = o[:, :, rows]
+    return o, exact, sim, (q, k, v, pos, ws)
+
+
+def test_prologue_matches_oracle_quantiser():
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2)
+    q, k, v, pos, cos, sin = _inputs(w, N=1000, seed=3)
+    B, H, N, d = q.shape
+    ws = dit.attention_workspace(B, H, N, d, precision="fp8", device=DEV)
+    dit.attention(q, k, v, cos, sin, precision="fp8", workspace=ws)
+    views = dit.fp8_workspace_views(ws, B, H, N, d)
+    qr = R.apply(q.cpu().double().numpy(), pos, w.axes)
+    kr = R.apply(k.cpu().double().numpy(), pos, w.axes)
+    mean = kr.mean(axis=2)
+    np.testing.assert_allclose(views["k_mean"].cpu().numpy(), mean, rtol=1e-4, atol=1e-4)
+    ks = F.smooth_k(kr)
+    for name, x, blk in (("q", qr, 128), ("k", ks, 64), ("v", v.cpu().double().numpy(), 64)):
+        codes, sc = F.quantize_blocks(x, blk)
+        np.testing.assert_allclose(views[name + "_scale"].cpu().double().numpy(), sc, rtol=2e-5)
+        got = views[name + "8"].cpu().view(torch.float8_e4m3fn).double().numpy()
+        # same value except where fp32 rotation/scaling lands on the other side of a rounding point
+        diff = got != codes
+        assert diff.mean() < 0.01, diff.mean()
+        step = np.abs(got - codes)[diff] / np.maximum(np.abs(codes[diff]), 2.0 ** -6)
+        assert (step <= 0.126).all()
+    np.testing.assert_allclose(views["v_scale_max"].cpu().numpy(), views["v_scale"].cpu().numpy().max(axis=2))
+
+
+@pytest.mark.parametrize("name,N", [("tiny", None), ("tiny", 129), ("tiny", 1000)])
+def test_fp8_tiny_d64_is_unsupported(name, N):
+    w = synth.WORKLOADS[name]
+    q, k, v, pos, cos, sin = _inputs(w, N)
+    with pytest.raises(dit.DitError):
+        dit.attention(q, k, v, cos, sin, precision="fp8")
+
+
+@pytest.mark.parametrize("N", [1, 64, 65, 129, 700, 4608])
+def test_fp8_normal_inputs_meet_target(N):
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2, outliers=False)
+    o, exact, sim, _ = _run(w, N=N, seed=N)
+    assert _cos(o, exact) >= 0.995, _cos(o, exact)
+    assert _cos(o, sim) >= 0.999, _cos(o, sim)
+
+
+def test_fp8_outlier_workload_matches_quantisation_floor():
+    w = synth.WORKLOADS["flux1k"]
+    rows = np.unique(np.concatenate([np.arange(0, 128), np.random.default_rng(4).integers(0, w.N, 256)]))
+    o, exact, sim, _ = _run(w, rows=rows)
+    floor = _cos(sim, exact)
+    got = _cos(o, exact)
+    assert _cos(o, sim) >= 0.999, _cos(o, sim)
+    assert got >= floor - 0.005, (got, floor)
+
+
+def test_fp8_bench_configuration_sampled_rows():
+    w = synth.WORKLOADS["flux2k"]
+    rows = np.unique(np.concatenate([np.arange(16896 - 64, 16896), np.random.default_rng(5).integers(0, w.N, 128)]))
+    o, exact, sim, _ = _run(w, rows=rows)
+    assert _cos(o, sim) >= 0.999, _cos(o, sim)
+    assert _cos(o, exact) >= _cos(sim, exact) - 0.005
+
+
+def test_fp8_smoothing_matters_for_shifted_keys():
+    """K with a +4 bias on the outlier channels: smoothing recovers the unshifted accuracy."""
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2)
+    q, k, v = synth.qkv(w, device=DEV, N=1024, seed=9, k_bias=4.0)
+    pos = synth.positions(w.T, 23)[:1024]
+    cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    exact = A.attention(q.cpu(), k.cpu(), v.cpu(), pos=pos.numpy(), axes=w.axes)
+    on = dit.attention(q, k, v, cos, sin, precision="fp8", smooth_k=True).cpu().double().numpy()
+    off = dit.attention(q, k, v, cos, sin, precision="fp8", smooth_k=False).cpu().double().numpy()
+    assert _cos(on, exact) >= _cos(off, exact) - 1e-3

@@ -118,6 +118,31 @@ def test_rope_is_applied_to_q_and_k_not_v():
                                A.attention(qr, kr, v), atol=1e-13)
 
 
+def test_round_bf16_matches_torch_cast_of_float32():
+    """fp32 -> bf16 in torch is a single round-to-nearest-even: an independent check."""
+    x = np.concatenate([rng.standard_normal(50000) * s for s in (1e-3, 1.0, 37.0, 1e4)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(A.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_round_bf16_ties_and_exact_values():
+    # 1 + 2^-8 is half-way between 1 and 1 + 2^-7: ties to even (1.0)
+    assert A.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert A.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2 * 2.0 ** -7
+    assert A.round_bf16(-3.0) == -3.0 and A.round_bf16(0.0) == 0.0
+
+
+def test_bf16_operand_reading_is_rounded_rotation():
+    w = synth.WORKLOADS["tiny"]
+    pos = synth.positions(w.T, w.G).numpy()
+    q, k, v = (rng.standard_normal((1, 1, w.N, 64)) for _ in range(3))
+    from oracle import rope
+    qr = A.round_bf16(rope.apply(q, pos, w.axes))
+    kr = A.round_bf16(rope.apply(k, pos, w.axes))
+    np.testing.assert_allclose(A.attention(q, k, v, pos=pos, axes=w.axes, operands="bf16"),
+                               A.attention(qr, kr, v), atol=1e-14)
+
+
 @pytest.mark.parametrize("mutation", ["no_scale", "transpose_v", "no_max_sub_row", "sum_over_queries"])
 def test_pins_catch_planted_mistakes(mutation):
     """Plant plausible mistakes in a copy of the oracle's formula and check a pin fails."""
