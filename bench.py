@@ -58,6 +58,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def gather_floats(x: float, world: int, device=None):
+    """Every rank's value of x, in rank order (one all_gather; CPU tensors under gloo)."""
+    if world == 1:
+        return [float(x)]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    out = [torch.zeros_like(t) for _ in range(world)]
+    dist.all_gather(out, t)
+    return [float(z.item()) for z in out]
+
+
 def aggregate(elapsed_ms_per_rank, units_per_rank, steps):
     """Whole-job throughput: all ranks' units over the slowest rank's time."""
     t = max(elapsed_ms_per_rank)
@@ -82,7 +94,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -233,12 +245,7 @@ def run_ours(args, rank, world, local_rank):
         return e0.elapsed_time(e1)
 
     def max_over_ranks(x):
-        if world == 1:
-            return [x]
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        out = [torch.zeros_like(t) for _ in range(world)]
-        dist.all_gather(out, t)
-        return [float(z.item()) for z in out]
+        return gather_floats(x, world, dev)
 
     # ---- main timed region: BF16 step (rotary + attention + gate)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
@@ -302,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
         ho.copy_(out, non_blocking=True)
         hskip.copy_(flag, non_blocking=True)
 
-    ke = max(3, min(args.steps, 10))
+    ke = max(3, min(args.steps, 20))
     ms_e2e = timed(step_e2e, ke, 2)
     all_e2e = max_over_ranks(ms_e2e)
     e2e_val, _ = aggregate(all_e2e, [flops * ke] * world, ke)
@@ -352,8 +359,8 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -31,6 +31,7 @@ constexpr int BN = 128;  // keys per tile
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold (log2 units)
 
 template <int D>
 struct Cfg {
@@ -38,7 +39,7 @@ struct Cfg {
   static constexpr int kTileBytes = BN * D * 2;           // one K or V tile (bf16)
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kSubTile = BN * 128;               // [rows][64] bf16 sub-tile (128-byte rows)
-  static constexpr int kNumBars = 1 + 3 * NST + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 3 * NST + 2 + 2 + 2;
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kQBytes + 2 * NST * kTileBytes + kNumBars * 8 + 16;
 };
 
@@ -49,7 +50,7 @@ struct Bars {
   uint64_t* kv_empty;
   uint64_t* s_full;   // [2]
   uint64_t* p_ready;  // [2]
-  uint64_t* pv_done;  // [1]
+  uint64_t* pv_done;  // [2]: PV(j) arrives on pv_done[j & 1]
 };
 
 template <int D>
@@ -91,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bars.s_full + s, 1);
       mbar_init(bars.p_ready + s, 128);
+      mbar_init(bars.pv_done + s, 1);
     }
-    mbar_init(bars.pv_done, 1);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ts(tO, tmem + ((jj & 1) ? kColP1 : kColP0) + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, C::kSubTile, 1024), idesc_o,
                        (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bars.pv_done);
+          mma_commit(bars.pv_done + (jj & 1));
           mma_commit(bars.kv_empty + st);
         }
       }
@@ -195,13 +196,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN; ++c)
           if (kv0 + c >= N) s[c] = 0xff800000u;  // -inf: key beyond the sequence
       }
-      float mx = __uint_as_float(s[0]);
+      // row max of the raw scores: 8 independent chains, then a tree
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-      const float m_new = fmaxf(m, mx * sl2);
-      const float alpha = ex2(m - m_new);
+      for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(s[i]);
+#pragma unroll
+      for (int c = 8; c < BN; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], __uint_as_float(s[c + i]));
+      const float m_tile =
+          fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])), fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+          sl2;
+      // Lazy rescale: the running max moves (and O is rescaled) only when some row of
+      // the warp gains more than kRescaleLog2; otherwise the stale max is kept, every
+      // p stays <= 2^kRescaleLog2 and O, l remain consistent, so the result is exact.
+      const bool grow = __any_sync(0xffffffffu, m_tile > m + kRescaleLog2);
+      const float m_new = grow ? fmaxf(m, m_tile) : m;
+      const float alpha = grow ? ex2(m - m_new) : 1.f;
       const float neg_m = -m_new;
-      float sum = 0.f;
+      // P(j) goes to buffer j&1, last read by PV(j-2)
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done + bsel, ((j >> 1) - 1) & 1, err, kErrTimeout));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const uint32_t tP = tmem + (bsel ? kColP1 : kColP0) + lane_off;
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
@@ -210,27 +229,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * e]), sl2, neg_m));
           const float p1 = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * e + 1]), sl2, neg_m));
-          sum += p0 + p1;
+          sum8[e & 7] += p0 + p1;
           p[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tP + c * 16, p);
       }
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done, (j - 1) & 1, err, kErrTimeout));
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      if (j > 0 && grow) {
+        // O holds PV(0..j-1) only once PV(j-1) has completed
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done + (bsel ^ 1), ((j - 1) >> 1) & 1, err, kErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint32_t tO = tmem + kColO + lane_off;
+        const uint32_t tO = tmem + kColO + lane_off;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-            reg_fence(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          reg_fence(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + c * 32, o);
         }
       }
       l = l * alpha + sum;
@@ -240,13 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bars.p_ready + bsel);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done, (nkv - 1) & 1, err, kErrTimeout));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.pv_done + ((nkv - 1) & 1), ((nkv - 1) >> 1) & 1, err, kErrTimeout));
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int grow = qt * BM + row;
+      const int qrow = qt * BM + row;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out.o) + b * out.so[0] + h * out.so[1] +
-                            static_cast<int64_t>(grow) * out.so[2];
+                            static_cast<int64_t>(qrow) * out.so[2];
       const uint32_t tO = tmem + kColO + lane_off;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -254,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         reg_fence(o);
-        if (grow < N) {
+        if (qrow < N) {
           uint4 pk[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll

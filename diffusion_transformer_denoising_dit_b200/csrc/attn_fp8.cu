@@ -31,7 +31,8 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 416;
 constexpr int kTileBytes = BN * D;  // e4m3: one byte per element, one 128-byte row per token
-constexpr int kNumBars = 1 + 3 * NST + 2 + 2 + 1;
+constexpr int kNumBars = 1 + 3 * NST + 2 + 2 + 2;
+constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold (log2 units)
 constexpr int kSmemBytes = 1024 + kTileBytes /*Q*/ + 2 * NST * kTileBytes + kNumBars * 8 + 16;
 
 struct Fp8Scales {
@@ -63,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_empty = v_full + NST;
   uint64_t* s_full = kv_empty + NST;
   uint64_t* p_ready = s_full + 2;
-  uint64_t* pv_done = p_ready + 2;
+  uint64_t* pv_done = p_ready + 2;  // [2]: PV(j) arrives on pv_done[j & 1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + kNumBars);
 
   const int warp = threadIdx.x >> 5;
@@ -83,8 +84,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
       mbar_init(p_ready + s, 128);
+      mbar_init(pv_done + s, 1);
     }
-    mbar_init(pv_done, 1);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = 32 rows of 128 bytes; P: 8 columns of 4 e4m3
             mma_f8_ts(tO, tmem + ((jj & 1) ? kColP1 : kColP0) + kk * 8,
                       smem_desc_sw128(v_addr + kk * 32 * 128, 16384, 1024), idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(pv_done);
+          mma_commit(pv_done + (jj & 1));
           mma_commit(kv_empty + st);
         }
       }
@@ -182,18 +183,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN; ++c)
           if (kv0 + c >= N) s[c] = 0xff800000u;
       }
-      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[64]);
+      // per-half row max of the raw scores: 4 independent chains per half
+      float mxa[4], mxb[4];
 #pragma unroll
-      for (int c = 1; c < 64; ++c) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[64 + c]));
+      for (int i = 0; i < 4; ++i) {
+        mxa[i] = __uint_as_float(s[i]);
+        mxb[i] = __uint_as_float(s[64 + i]);
       }
+#pragma unroll
+      for (int c = 4; c < 64; c += 4)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mxa[i] = fmaxf(mxa[i], __uint_as_float(s[c + i]));
+          mxb[i] = fmaxf(mxb[i], __uint_as_float(s[64 + c + i]));
+        }
+      const float mx0 = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+      const float mx1 = fmaxf(fmaxf(mxb[0], mxb[1]), fmaxf(mxb[2], mxb[3]));
       // c0, c1 > 0 for every in-range block; a block past the end is all -inf
       const float m_tile = fmaxf(mx0 * c0, kv0 + 64 < N ? mx1 * c1 : -INFINITY);
-      const float m_new = fmaxf(m, m_tile);
-      const float alpha = ex2(m - m_new);
+      // lazy rescale (see the BF16 kernel): exact, the stale max bounds p by 2^kRescaleLog2
+      const bool grow = __any_sync(0xffffffffu, m_tile > m + kRescaleLog2);
+      const float m_new = grow ? fmaxf(m, m_tile) : m;
+      const float alpha = grow ? ex2(m - m_new) : 1.f;
       const float neg_m = -m_new;
-      float sum = 0.f;
+      if (j >= 2) {  // P(j) goes to buffer j&1, last read by PV(j-2)
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done + bsel, ((j >> 1) - 1) & 1, err, kErrTimeout));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t tP = tmem + (bsel ? kColP1 : kColP0) + lane_off;
       uint32_t p[32];
 #pragma unroll
@@ -204,27 +222,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           x[i] = ex2(fmaf(__uint_as_float(s[4 * e + i]), cs, neg_m));
-          sum += x[i];
+          sum4[i] += x[i];
         }
         p[e] = cvt_e4m3x4(x[0] * fv, x[1] * fv, x[2] * fv, x[3] * fv);
       }
       tmem_st32(tP, p);
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, err, kErrTimeout));
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (j > 0 && grow) {
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done + (bsel ^ 1), ((j - 1) >> 1) & 1, err, kErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint32_t tO = tmem + kColO + lane_off;
+        const uint32_t tO = tmem + kColO + lane_off;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-            reg_fence(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          reg_fence(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + c * 32, o);
         }
       }
       l = l * alpha + sum;
@@ -233,13 +250,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_ready + bsel);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (nkv - 1) & 1, err, kErrTimeout));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((nkv - 1) & 1), ((nkv - 1) >> 1) & 1, err, kErrTimeout));
     if (ok) {
       tc_fence_after();
       const float fin = vmax / 448.f / l;
-      const int grow = qt * BM + row;
+      const int qrow = qt * BM + row;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out.o) + b * out.so[0] + h * out.so[1] +
-                            static_cast<int64_t>(grow) * out.so[2];
+                            static_cast<int64_t>(qrow) * out.so[2];
       const uint32_t tO = tmem + kColO + lane_off;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         reg_fence(o);
-        if (grow < N) {
+        if (qrow < N) {
           uint4 pk[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
