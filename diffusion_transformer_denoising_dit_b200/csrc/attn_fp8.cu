@@ -32,7 +32,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 416;
 constexpr int kTileBytes = BN * D;  // e4m3: one byte per element, one 128-byte row per token
 constexpr int kNumBars = 1 + 3 * NST + 2 + 2 + 2;
-constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold (log2 units)
+// P is quantised as p * 448 * sV/sV_max with p <= 2^kRescaleLog2, so e4m3's range
+// (max 448) leaves no headroom for a stale max: rescale whenever the max grows.
+constexpr float kRescaleLog2 = 0.f;
 constexpr int kSmemBytes = 1024 + kTileBytes /*Q*/ + 2 * NST * kTileBytes + kNumBars * 8 + 16;
 
 struct Fp8Scales {
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mx1 = fmaxf(fmaxf(mxb[0], mxb[1]), fmaxf(mxb[2], mxb[3]));
       // c0, c1 > 0 for every in-range block; a block past the end is all -inf
       const float m_tile = fmaxf(mx0 * c0, kv0 + 64 < N ? mx1 * c1 : -INFINITY);
-      // lazy rescale (see the BF16 kernel): exact, the stale max bounds p by 2^kRescaleLog2
+      // rescale whenever some row of the warp gets a larger max (kRescaleLog2 = 0)
       const bool grow = __any_sync(0xffffffffu, m_tile > m + kRescaleLog2);
       const float m_new = grow ? fmaxf(m, m_tile) : m;
       const float alpha = grow ? ex2(m - m_new) : 1.f;

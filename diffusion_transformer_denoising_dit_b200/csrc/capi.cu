@@ -10,7 +10,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/dit.h"
+#include "dit.h"
 #include "dit_internal.h"
 
 namespace {
