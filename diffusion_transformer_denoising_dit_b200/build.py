@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdit.so")
 SOURCES = ["capi.cu", "rope.cu", "gate.cu", "attn_bf16.cu", "attn_fp8.cu", "fp8_prologue.cu"]
-HEADERS = ["dit_device.cuh", "dit_internal.h"]
+HEADERS = ["dit_device.cuh", "dit_internal.h", "attn_kernel.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

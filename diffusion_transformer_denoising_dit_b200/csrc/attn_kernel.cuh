@@ -1,0 +1,411 @@
+// Joint attention kernel for sm_100a, shared by the BF16 and FP8 variants:
+// TMA -> shared memory -> tcgen05 MMA -> TMEM, flash-style online softmax in
+// fp32 with exp2.
+//
+// Source: "FLUX 3 Image Klein / TensorRT-LLM VisualGen", section on why the
+// differences arise: the DiT's VANILLA BF16 attention over the joint
+// text+image tokens is about 60 % of its GPU kernel time, and cuDNN FP8
+// attention is its quantised counterpart.  O = softmax(scale Q K^T) V per
+// (batch, head), bidirectional over every key.
+//
+// One CTA owns two 128-row Q tiles (Q0, Q1) of one (b, h) and streams every
+// K/V tile of that head once for both, halving the K/V traffic from L2 per
+// FLOP compared with one tile per CTA.  320 threads:
+//   warps 0-3  softmax of Q0 (thread t = row t = TMEM lane t)
+//   warps 4-7  softmax of Q1
+//   warp 8     TMA producer: Q0, Q1 once; K_j into a NK-deep ring, V_j into a NV-deep ring
+//   warp 9     MMA issuer (one thread) and TMEM owner
+// TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256) O0, O1 (d
+// columns each from 256).  P_i (bf16: 64 columns, e4m3: 32) overwrites the
+// first columns of S_i once the softmax has read S_i.
+// The MMA thread issues, per key tile j:
+//     O0 += P0(j-1) V(j-1);  S0(j) = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1(j) = Q1 K(j)^T
+// tcgen05 MMAs from one thread execute in issue order, so S_i(j) never
+// overwrites P_i(j-1) before PV_i(j-1) has read it; and the commit that
+// signals S_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j), O_i
+// already holds every PV_i before j and may be rescaled in place.  The tensor
+// core thus runs PV1(j-1), S1(j) while softmax 0 works on S0(j), and PV0(j),
+// S0(j+1) while softmax 1 works on S1(j).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "dit_device.cuh"
+
+namespace dit {
+
+template <bool FP8, int D>
+struct AttnCfg {
+  static constexpr int BM = 128;                        // rows per Q tile (two per CTA)
+  static constexpr int BN = 128;                        // keys per K/V tile
+  static constexpr int kThreads = 320;
+  static constexpr int EB = FP8 ? 1 : 2;                // element bytes
+  static constexpr int kRowBytes = D * EB;              // bytes of one token row
+  static constexpr int kSub = kRowBytes / 128;          // 128-byte swizzle column blocks per row
+  static constexpr int kSubBytes = BN * 128;            // one [128 rows][128 B] column block
+  static constexpr int kTileBytes = BN * kRowBytes;     // one Q, K or V tile
+  static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
+  static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
+  static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 16;
+  static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
+  static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
+  static constexpr uint32_t kTmemCols = 512;
+  // lazy rescale threshold (log2 units): with a stale max every p <= 2^kRescaleLog2.
+  // e4m3 P (p * 448 * sV / sV_max) has no headroom for that, so FP8 rescales on any growth.
+  static constexpr float kRescaleLog2 = FP8 ? 0.f : 8.f;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kRowBytes % 128 == 0, "token rows must be whole 128-byte swizzle atoms");
+};
+
+// Scales of the FP8 variant (unused by BF16).
+struct AttnScales {
+  const float* q_scale;      // [B*H][nq]  (128-token blocks)
+  const float* k_scale;      // [B*H][nk]  (64-token blocks)
+  const float* v_scale;      // [B*H][nk]
+  const float* v_scale_max;  // [B*H]
+  int H;
+};
+
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+template <bool FP8, int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnOut out, const AttnScales sc) {
+  using C = AttnCfg<FP8, D>;
+  constexpr int NK = C::NK, NV = C::NV, BM = C::BM, BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                        // Q0, Q1
+  uint8_t* sK = sQ + 2 * C::kTileBytes;      // NK stages
+  uint8_t* sV = sK + NK * C::kTileBytes;     // NV stages
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(sV + NV * C::kTileBytes);  // [2]
+  uint64_t* k_full = q_full + 2;
+  uint64_t* k_empty = k_full + NK;
+  uint64_t* v_full = k_empty + NK;
+  uint64_t* v_empty = v_full + NV;
+  uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and PV_i(j-1) done)
+  uint64_t* p_ready = s_full + 2;    // [2] softmax i finished tile j (128 arrivals)
+  uint64_t* o_done = p_ready + 2;    // every MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int N = out.N;
+  const int nkv = (N + BN - 1) / BN;
+  int* err = out.err;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(p_ready + i, 128);
+    }
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    mbar_init(o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mbar_arrive_expect_tx(q_full + i, C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kSub; ++c)
+          tma_load_4d(sQ + i * C::kTileBytes + c * C::kSubBytes, &tmQ, q_full + i, c * C::kBoxInner,
+                      (2 * qt + i) * BM, h, b);
+      }
+      for (int j = 0; j < nkv; ++j) {
+        const int sk = j % NK, sv = j % NV;
+        if (j >= NK && !mbar_wait(k_empty + sk, ((j / NK) & 1) ^ 1, err, kErrTimeout)) break;
+        mbar_arrive_expect_tx(k_full + sk, C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kSub; ++c)
+          tma_load_4d(sK + sk * C::kTileBytes + c * C::kSubBytes, &tmK, k_full + sk, c * C::kBoxInner, j * BN, h, b);
+        if (j >= NV && !mbar_wait(v_empty + sv, ((j / NV) & 1) ^ 1, err, kErrTimeout)) break;
+        mbar_arrive_expect_tx(v_full + sv, C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kSub; ++c)
+          tma_load_4d(sV + sv * C::kTileBytes + c * C::kSubBytes, &tmV, v_full + sv, c * C::kBoxInner, j * BN, h, b);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = FP8 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
+      constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, BM, BN);  // Q, K both K-major
+      constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 1, BM, D);   // V MN-major (d contiguous)
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      auto qk = [&](int i, int sk) {  // S_i = Q_i K^T
+        const uint32_t qa = q_addr + i * C::kTileBytes, ka = k_addr + sk * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / C::kKStep; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;  // 32 bytes of K per MMA
+          const uint64_t ad = smem_desc_sw128(qa + off, 16, 1024), bd = smem_desc_sw128(ka + off, 16, 1024);
+          if constexpr (FP8)
+            mma_f8_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          else
+            mma_f16_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto pv = [&](int i, int sv, bool acc) {  // O_i (+)= P_i V
+        const uint32_t va = v_addr + sv * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / C::kKStep; ++kk) {
+          // kKStep keys = kKStep rows of 128 bytes; d column blocks are kSubBytes apart
+          const uint64_t bd = smem_desc_sw128(va + kk * C::kKStep * 128, C::kSubBytes, 1024);
+          const uint32_t pa = tmem + C::kColS + 128 * i + kk * 8;  // 8 columns of packed P per MMA
+          if constexpr (FP8)
+            mma_f8_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, err, kErrTimeout) && mbar_wait(k_full, 0, err, kErrTimeout);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        mma_commit(s_full);
+        ok = mbar_wait(q_full + 1, 0, err, kErrTimeout);
+      }
+      if (ok) {
+        tc_fence_after();
+        qk(1, 0);
+        mma_commit(s_full + 1);
+        mma_commit(k_empty);
+      }
+      for (int j = 1; ok && j <= nkv; ++j) {
+        const int jj = j - 1, sv = jj % NV, sk = j % NK;
+        if (!mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout)) break;
+        if (!mbar_wait(p_ready, jj & 1, err, kErrTimeout)) break;
+        tc_fence_after();
+        pv(0, sv, jj > 0);
+        if (j < nkv) {
+          if (!mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout)) break;
+          tc_fence_after();
+          qk(0, sk);
+          mma_commit(s_full);
+        }
+        if (!mbar_wait(p_ready + 1, jj & 1, err, kErrTimeout)) break;
+        tc_fence_after();
+        pv(1, sv, jj > 0);
+        mma_commit(v_empty + sv);
+        if (j < nkv) {
+          qk(1, sk);
+          mma_commit(s_full + 1);
+          mma_commit(k_empty + sk);
+        }
+      }
+      mma_commit(o_done);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int i = warp >> 2;                    // Q tile of this warpgroup
+    const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + C::kColS + 128 * i + lane_off;
+    const uint32_t tO = tmem + C::kColO + D * i + lane_off;
+    const float sl2 = out.scale_log2;
+    const int qblk = 2 * qt + i;                // 128-row block index of this Q tile
+    // FP8 scales: score = S * sQ * sK(j) * scale, P8 = p * 448 * sV(j) / sV_max
+    float qs = sl2, vfold = 1.f, fin_scale = 1.f;
+    const float* ksc = nullptr;
+    const float* vsc = nullptr;
+    int nk = 0;
+    if constexpr (FP8) {
+      const int bh = b * sc.H + h;
+      const int nq = (N + 127) / 128;
+      nk = (N + 63) / 64;
+      ksc = sc.k_scale + static_cast<int64_t>(bh) * nk;
+      vsc = sc.v_scale + static_cast<int64_t>(bh) * nk;
+      const float vmax = sc.v_scale_max[bh];
+      qs = (qblk < nq ? sc.q_scale[static_cast<int64_t>(bh) * nq + qblk] : 1.f) * sl2;
+      vfold = 448.f / vmax;
+      fin_scale = vmax / 448.f;
+    }
+    float m = -INFINITY;  // running (possibly stale) max of the scaled log2 scores
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, j & 1, err, kErrTimeout));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+      tmem_wait_ld();
+      reg_fence(s);
+      const int kv0 = j * BN;
+      if (kv0 + BN > N) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (kv0 + c >= N) s[c] = 0xff800000u;  // -inf: key beyond the sequence
+      }
+      // per-64-key-half score multipliers (both equal for BF16)
+      float c0 = sl2, c1 = sl2, f0 = 1.f, f1 = 1.f;
+      if constexpr (FP8) {
+        const int kb0 = 2 * j, kb1 = 2 * j + 1;
+        c0 = qs * ksc[kb0];
+        c1 = kb1 < nk ? qs * ksc[kb1] : 1.f;  // past the end every key is -inf; keep -inf * c1 = -inf
+        f0 = vsc[kb0] * vfold;
+        f1 = kb1 < nk ? vsc[kb1] * vfold : 0.f;
+      }
+      // row max: 4 independent chains per 64-key half, then a tree
+      float ma[4], mb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ma[e] = __uint_as_float(s[e]);
+        mb[e] = __uint_as_float(s[64 + e]);
+      }
+#pragma unroll
+      for (int c = 4; c < 64; c += 4)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          ma[e] = fmaxf(ma[e], __uint_as_float(s[c + e]));
+          mb[e] = fmaxf(mb[e], __uint_as_float(s[64 + c + e]));
+        }
+      const float mx0 = fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3]));
+      const float mx1 = fmaxf(fmaxf(mb[0], mb[1]), fmaxf(mb[2], mb[3]));
+      // the first key of a tile is always in range; a half past the end is all -inf
+      const float m_tile = fmaxf(mx0 * c0, kv0 + 64 < N ? mx1 * c1 : -INFINITY);
+      const bool grow = __any_sync(0xffffffffu, m_tile > m + C::kRescaleLog2);
+      const float m_new = grow ? fmaxf(m, m_tile) : m;
+      const float alpha = grow ? ex2(m - m_new) : 1.f;
+      const float neg_m = -m_new;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (FP8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // 32 keys -> 8 columns of 4 e4m3 each
+          uint32_t p[8];
+          const float cs = q < 2 ? c0 : c1;
+          const float fv = q < 2 ? f0 : f1;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              x[u] = ex2(fmaf(__uint_as_float(s[32 * q + 4 * e + u]), cs, neg_m));
+              sum4[u] += x[u];
+            }
+            p[e] = cvt_e4m3x4(x[0] * fv, x[1] * fv, x[2] * fv, x[3] * fv);
+          }
+          tmem_st8(tS + 8 * q, p);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 columns of 2 bf16 each
+          uint32_t p[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[32 * q + 2 * e]), sl2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(s[32 * q + 2 * e + 1]), sl2, neg_m));
+            sum4[e & 3] += p0 + p1;
+            p[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * q, p);
+        }
+      }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1): the commit behind s_full covered them
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      l = l * alpha + sum;
+      m = m_new;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_ready + i);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, 0, err, kErrTimeout));
+    if (ok) {
+      tc_fence_after();
+      const float fin = fin_scale / l;
+      const int qrow = qblk * BM + row;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out.o) + b * out.so[0] + h * out.so[1] +
+                            static_cast<int64_t>(qrow) * out.so[2];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        if (qrow < N) {
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * fin, __uint_as_float(o[2 * e + 1]) * fin);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <bool FP8, int D>
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
+                        const AttnScales& sc, int B, int H, cudaStream_t stream) {
+  constexpr int smem = AttnCfg<FP8, D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<FP8, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((out.N + 255) / 256, H, B);
+  attn_kernel<FP8, D><<<grid, AttnCfg<FP8, D>::kThreads, smem, stream>>>(tq, tk, tv, out, sc);
+  return cudaGetLastError();
+}
+
+}  // namespace dit
