@@ -10,22 +10,29 @@
 //
 // One CTA owns two 128-row Q tiles (Q0, Q1) of one (b, h) and streams every
 // K/V tile of that head once for both, halving the K/V traffic from L2 per
-// FLOP compared with one tile per CTA.  320 threads:
+// FLOP compared with one tile per CTA.  384 threads:
 //   warps 0-3  softmax of Q0 (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax of Q1
 //   warp 8     TMA producer: Q0, Q1 once; K_j into a NK-deep ring, V_j into a NV-deep ring
 //   warp 9     MMA issuer (one thread) and TMEM owner
+//   warps 10-11 idle (they complete the third warpgroup for the register re-split)
+// Registers: launched at 168 per thread; the third warpgroup drops to kRegsAux and
+// the softmax warpgroups rise to kRegsSoftmax (2*128*kRegsSoftmax + 128*kRegsAux <= 64K).
 // TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256) O0, O1 (d
 // columns each from 256).  P_i (bf16: 64 columns, e4m3: 32) overwrites the
 // first columns of S_i once the softmax has read S_i.
 // The MMA thread issues, per key tile j:
 //     O0 += P0(j-1) V(j-1);  S0(j) = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1(j) = Q1 K(j)^T
-// tcgen05 MMAs from one thread execute in issue order, so S_i(j) never
-// overwrites P_i(j-1) before PV_i(j-1) has read it; and the commit that
-// signals S_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j), O_i
-// already holds every PV_i before j and may be rescaled in place.  The tensor
-// core thus runs PV1(j-1), S1(j) while softmax 0 works on S0(j), and PV0(j),
-// S0(j+1) while softmax 1 works on S1(j).
+// tcgen05 MMAs from one thread are executed in issue order, so S_i(j) never
+// overwrites P_i(j-1) before PV_i(j-1) has read it.  Completion is signalled
+// per dependency, never inferred from a later commit: a commit right after
+// PV_i arrives on pv_done[i] (softmax i waits for it before touching O_i);
+// K and V stages are freed by count-2 barriers that get one commit after each
+// of the two MMAs reading the stage.  (Measured: relying on the commit behind
+// S_i(j) to cover PV_i(j-1) made the O rescale race.)  The tensor core runs
+// PV1(j-1), S1(j) while softmax 0 works on S0(j), and PV0(j), S0(j+1) while
+// softmax 1 works on S1(j); the two softmax warpgroups take turns on the ex2
+// unit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -38,7 +45,9 @@ template <bool FP8, int D>
 struct AttnCfg {
   static constexpr int BM = 128;                        // rows per Q tile (two per CTA)
   static constexpr int BN = 128;                        // keys per K/V tile
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegsSoftmax = 208, kRegsAux = 80;
+  static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= 65536, "register re-split exceeds the register file");
   static constexpr int EB = FP8 ? 1 : 2;                // element bytes
   static constexpr int kRowBytes = D * EB;              // bytes of one token row
   static constexpr int kSub = kRowBytes / 128;          // 128-byte swizzle column blocks per row
@@ -47,7 +56,7 @@ struct AttnCfg {
   static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
   static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
   static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2;
   static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 16;
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
@@ -82,7 +91,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 }
 
 template <bool FP8, int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnOut out, const AttnScales sc) {
   using C = AttnCfg<FP8, D>;
@@ -97,9 +106,10 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* k_empty = k_full + NK;
   uint64_t* v_full = k_empty + NK;
   uint64_t* v_empty = v_full + NV;
-  uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and PV_i(j-1) done)
+  uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed
   uint64_t* p_ready = s_full + 2;    // [2] softmax i finished tile j (128 arrivals)
-  uint64_t* o_done = p_ready + 2;    // every MMA done
+  uint64_t* pv_done = p_ready + 2;   // [2] PV_i(j) computed
+  uint64_t* turn = pv_done + 2;      // [2] softmax i may exponentiate (ping-pong between the warpgroups)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
 
   const int warp = threadIdx.x >> 5;
@@ -114,16 +124,17 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(q_full + i, 1);
       mbar_init(s_full + i, 1);
       mbar_init(p_ready + i, 128);
+      mbar_init(pv_done + i, 1);
+      mbar_init(turn + i, 128);
     }
     for (int s = 0; s < NK; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(k_empty + s, 1);
+      mbar_init(k_empty + s, 2);  // one commit after each of S0, S1
     }
     for (int s = 0; s < NV; ++s) {
       mbar_init(v_full + s, 1);
-      mbar_init(v_empty + s, 1);
+      mbar_init(v_empty + s, 2);  // one commit after each of PV0, PV1
     }
-    mbar_init(o_done, 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -135,7 +146,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+   regs_dec<C::kRegsAux>();
+   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -202,6 +215,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         qk(0, 0);
         mma_commit(s_full);
+        mma_commit(k_empty);
         ok = mbar_wait(q_full + 1, 0, err, kErrTimeout);
       }
       if (ok) {
@@ -216,15 +230,19 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(p_ready, jj & 1, err, kErrTimeout)) break;
         tc_fence_after();
         pv(0, sv, jj > 0);
+        mma_commit(pv_done);
+        mma_commit(v_empty + sv);
         if (j < nkv) {
           if (!mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout)) break;
           tc_fence_after();
           qk(0, sk);
           mma_commit(s_full);
+          mma_commit(k_empty + sk);
         }
         if (!mbar_wait(p_ready + 1, jj & 1, err, kErrTimeout)) break;
         tc_fence_after();
         pv(1, sv, jj > 0);
+        mma_commit(pv_done + 1);
         mma_commit(v_empty + sv);
         if (j < nkv) {
           qk(1, sk);
@@ -232,9 +250,10 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(k_empty + sk);
         }
       }
-      mma_commit(o_done);
     }
+   }
   } else {
+    regs_inc<C::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     const int i = warp >> 2;                    // Q tile of this warpgroup
     const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
@@ -264,6 +283,8 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, j & 1, err, kErrTimeout));
+      // PV_i(j-1) done: O_i may be rescaled (consumed every tile, so phases stay in step)
+      if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, (j - 1) & 1, err, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[BN];
@@ -286,82 +307,103 @@ __global__ void __launch_bounds__(320, 1)
         f0 = vsc[kb0] * vfold;
         f1 = kb1 < nk ? vsc[kb1] * vfold : 0.f;
       }
-      // row max: 4 independent chains per 64-key half, then a tree
-      float ma[4], mb[4];
+      // row max: two 3-input max chains per 64-key half
+      float ma0 = __uint_as_float(s[0]), ma1 = __uint_as_float(s[1]);
+      float mb0 = __uint_as_float(s[64]), mb1 = __uint_as_float(s[65]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        ma[e] = __uint_as_float(s[e]);
-        mb[e] = __uint_as_float(s[64 + e]);
+      for (int c = 2; c < 64; c += 4) {
+        ma0 = fmax3(ma0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        ma1 = fmax3(ma1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        mb0 = fmax3(mb0, __uint_as_float(s[64 + c]), __uint_as_float(s[64 + c + 1]));
+        mb1 = fmax3(mb1, __uint_as_float(s[64 + c + 2]), __uint_as_float(s[64 + c + 3]));
       }
-#pragma unroll
-      for (int c = 4; c < 64; c += 4)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          ma[e] = fmaxf(ma[e], __uint_as_float(s[c + e]));
-          mb[e] = fmaxf(mb[e], __uint_as_float(s[64 + c + e]));
-        }
-      const float mx0 = fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3]));
-      const float mx1 = fmaxf(fmaxf(mb[0], mb[1]), fmaxf(mb[2], mb[3]));
+      const float mx0 = fmaxf(ma0, ma1);
+      const float mx1 = fmaxf(mb0, mb1);
       // the first key of a tile is always in range; a half past the end is all -inf
       const float m_tile = fmaxf(mx0 * c0, kv0 + 64 < N ? mx1 * c1 : -INFINITY);
       const bool grow = __any_sync(0xffffffffu, m_tile > m + C::kRescaleLog2);
       const float m_new = grow ? fmaxf(m, m_tile) : m;
       const float alpha = grow ? ex2(m - m_new) : 1.f;
-      const float neg_m = -m_new;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (FP8) {
+      // Ping-pong: the two warpgroups take turns on the ex2 unit, so one exponentiates
+      // while the other's PV and next S run on the tensor core.  Softmax 0 goes first in
+      // every tile; softmax 1 starts tile j once softmax 0 has finished tile j's exps.
+      if (i == 1 || j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(turn + i, (i == 1 ? j : j - 1) & 1, err, kErrTimeout));
+        if (!ok) break;
+      }
+      // p = 2^(s * c - m): packed scale-and-subtract, ex2 per element, packed row
+      // sums in 4 chains (in the shadow of the ex2 pipe), P to TMEM per 32 keys.
+      // tcgen05.st reads its source registers asynchronously: every register a
+      // pending store reads stays pinned (reg_fence after tcgen05.wait::st) so the
+      // compiler cannot reuse it before the store has completed.
+      const uint64_t nm2 = f2(-m_new, -m_new);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      constexpr int kPRegs = FP8 ? 32 : 64;  // packed P of the whole row
+      uint32_t p[kPRegs];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 32 keys -> 8 columns of 4 e4m3 each
-          uint32_t p[8];
-          const float cs = q < 2 ? c0 : c1;
-          const float fv = q < 2 ? f0 : f1;
+      for (int q = 0; q < 4; ++q) {  // 32 keys per TMEM store
+        const uint64_t cq = FP8 ? (q < 2 ? f2(c0, c0) : f2(c1, c1)) : f2(sl2, sl2);
+        if constexpr (FP8) {  // 32 keys -> 8 columns of 4 e4m3 (V block scale folded in)
+          const uint64_t fv = q < 2 ? f2(f0, f0) : f2(f1, f1);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            float x[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              x[u] = ex2(fmaf(__uint_as_float(s[32 * q + 4 * e + u]), cs, neg_m));
-              sum4[u] += x[u];
-            }
-            p[e] = cvt_e4m3x4(x[0] * fv, x[1] * fv, x[2] * fv, x[3] * fv);
+            const int k0 = 32 * q + 4 * e;
+            float x0, x1, x2, x3;
+            f2_split(ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), cq, nm2), x0, x1);
+            f2_split(ffma2(f2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), cq, nm2), x2, x3);
+            const uint64_t pa = f2(ex2(x0), ex2(x1)), pb = f2(ex2(x2), ex2(x3));
+            acc[(2 * e) & 3] = fadd2(acc[(2 * e) & 3], pa);
+            acc[(2 * e + 1) & 3] = fadd2(acc[(2 * e + 1) & 3], pb);
+            float a, bq, cc, dd;
+            f2_split(fmul2(pa, fv), a, bq);
+            f2_split(fmul2(pb, fv), cc, dd);
+            p[8 * q + e] = cvt_e4m3x4(a, bq, cc, dd);
           }
-          tmem_st8(tS + 8 * q, p);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 columns of 2 bf16 each
-          uint32_t p[16];
+          tmem_st8(tS + 8 * q, p + 8 * q);
+        } else {  // 32 keys -> 16 columns of 2 bf16
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[32 * q + 2 * e]), sl2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(s[32 * q + 2 * e + 1]), sl2, neg_m));
-            sum4[e & 3] += p0 + p1;
-            p[e] = pack_bf16x2(p0, p1);
+            float x, y;
+            f2_split(ffma2(f2(__uint_as_float(s[32 * q + 2 * e]), __uint_as_float(s[32 * q + 2 * e + 1])), cq, nm2), x,
+                     y);
+            const float p0 = ex2(x), p1 = ex2(y);
+            acc[e & 3] = fadd2(acc[e & 3], f2(p0, p1));
+            p[16 * q + e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tS + 16 * q, p);
+          tmem_st16(tS + 16 * q, p + 16 * q);
         }
       }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1): the commit behind s_full covered them
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          reg_fence(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + c * 32, o);
-        }
-      }
-      l = l * alpha + sum;
-      m = m_new;
+      mbar_arrive(turn + (i ^ 1));
       tmem_wait_st();
+      reg_fence(p);
+      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1) (pv_done waited above)
+        uint32_t o[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o + c * 32);
+        tmem_wait_ld();
+        reg_fence(o);
+        const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll
+        for (int e = 0; e < D / 2; ++e) {
+          float x, y;
+          f2_split(fmul2(f2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), a2), x, y);
+          o[2 * e] = __float_as_uint(x);
+          o[2 * e + 1] = __float_as_uint(y);
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_st32(tO + c * 32, o + c * 32);
+        tmem_wait_st();
+        reg_fence(o);
+      }
       tc_fence_before();
       mbar_arrive(p_ready + i);
+      float a0, a1;
+      f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+      l = l * alpha + (a0 + a1);
+      m = m_new;
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, 0, err, kErrTimeout));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, (nkv - 1) & 1, err, kErrTimeout));
     if (ok) {
       tc_fence_after();
       const float fin = fin_scale / l;
