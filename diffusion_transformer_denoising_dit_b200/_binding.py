@@ -19,7 +19,7 @@ STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "D
           4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT"}
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
-           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate"]
+           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc"]
 
 
 class DitError(RuntimeError):
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.fbcache_gate_workspace_bytes.argtypes = [ctypes.c_int64]
         L.fbcache_gate.restype = _i
         L.fbcache_gate.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+        L.fbcache_gate_noalloc.restype = _i
+        L.fbcache_gate_noalloc.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp]
         _lib = L
     return _lib
 

@@ -14,6 +14,9 @@
 // tree order, so the result is deterministic for a given n.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
+#include "dit.h"
 #include "dit_device.cuh"
 
 namespace dit {
@@ -131,3 +134,69 @@ cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold
 }
 
 }  // namespace dit
+
+// ---------------------------------------------------------------------------
+// fbcache_gate_noalloc: the same two-pass gate, with its scratch in a fixed
+// device array instead of a caller-provided workspace.
+//
+// For callers that cannot hand this library any device memory: a plug-in
+// driven by a host runtime that owns the device allocator and exposes no
+// scratch buffers, or a step loop whose rules forbid allocating while it runs.
+// The scratch holds one (sum|a-b|, sum|b|) pair of doubles per pass-1 CTA.
+// Pass 1 writes every pair that pass 2 reads, so nothing has to start at zero.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Largest scratch any n can need: 2 doubles for each of at most kGateMaxCtas CTAs.
+constexpr int kNoAllocScratchDoubles = 2 * dit::kGateMaxCtas;
+static __device__ __align__(256) double g_gate_scratch[kNoAllocScratchDoubles];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+double* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device (looked up once per device).
+double* noalloc_scratch(dit_status* st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    *st = DIT_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) {
+      *st = DIT_ERR_UNSUPPORTED;
+      return nullptr;
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gate_scratch) != cudaSuccess || p == nullptr) {
+      *st = DIT_ERR_LAUNCH;
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = static_cast<double*>(p);
+  }
+  *st = DIT_OK;
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" DIT_API dit_status fbcache_gate_noalloc(const void* r_cur, const void* r_prev, int64_t n, float threshold,
+                                                   float* rel_out, int32_t* skip_out, dit_stream_t stream) {
+  if (!r_cur || !r_prev || !rel_out || !skip_out || n < 1) return DIT_ERR_INVALID_ARG;
+  if (!(threshold == threshold) || threshold > 3.4e38f || threshold < -3.4e38f) return DIT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(r_cur) & 15u) || (reinterpret_cast<uintptr_t>(r_prev) & 15u))
+    return DIT_ERR_ALIGNMENT;
+  // the fixed array must hold every pass-1 partial for this n
+  if (2 * static_cast<int64_t>(dit::gate_num_ctas(n)) > kNoAllocScratchDoubles) return DIT_ERR_WORKSPACE;
+  dit_status st;
+  double* scratch = noalloc_scratch(&st);
+  if (!scratch) return st;
+  return dit::launch_gate(r_cur, r_prev, n, threshold, rel_out, skip_out, scratch,
+                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DIT_OK
+             : DIT_ERR_LAUNCH;
+}

@@ -151,6 +151,23 @@ DIT_API size_t fbcache_gate_workspace_bytes(int64_t n);
 DIT_API dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float threshold, float* rel_out,
                         int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream);
 
+/* fbcache_gate without a workspace argument (the pages have no counterpart:
+ * this is a convenience of this library).  For callers that cannot give the
+ * library device memory, e.g. a plug-in run by a host framework that owns the
+ * device allocator, or a step loop that must not allocate while it runs.
+ * Same inputs, outputs, arithmetic and result as fbcache_gate; its scratch
+ * is a fixed device array of 2 * 1184 doubles (18,944 bytes) inside the
+ * library, held by every device that loads it until the process exits.
+ * Limit: the scratch must hold 2 doubles per pass-1 CTA; the CTA count is
+ * capped at 1184 for any n, so every n >= 1 fits (a larger need would return
+ * DIT_ERR_WORKSPACE).  Nothing in the array has to start at zero.  The first
+ * call on a device looks up the array's device address (a runtime query), so
+ * make that first call before capturing the stream.  All calls share the one
+ * array: calls that overlap on the GPU (different streams without ordering)
+ * race on it; calls on one stream are safe. */
+DIT_API dit_status fbcache_gate_noalloc(const void* r_cur, const void* r_prev, int64_t n, float threshold,
+                                        float* rel_out, int32_t* skip_out, dit_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
