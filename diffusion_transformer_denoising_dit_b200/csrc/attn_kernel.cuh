@@ -24,15 +24,16 @@
 // The MMA thread issues, per key tile j:
 //     O0 += P0(j-1) V(j-1);  S0(j) = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1(j) = Q1 K(j)^T
 // tcgen05 MMAs from one thread are executed in issue order, so S_i(j) never
-// overwrites P_i(j-1) before PV_i(j-1) has read it.  Completion is signalled
-// per dependency, never inferred from a later commit: a commit right after
-// PV_i arrives on pv_done[i] (softmax i waits for it before touching O_i);
-// K and V stages are freed by count-2 barriers that get one commit after each
-// of the two MMAs reading the stage.  (Measured: relying on the commit behind
-// S_i(j) to cover PV_i(j-1) made the O rescale race.)  The tensor core runs
-// PV1(j-1), S1(j) while softmax 0 works on S0(j), and PV0(j), S0(j+1) while
-// softmax 1 works on S1(j); the two softmax warpgroups take turns on the ex2
-// unit.
+// overwrites P_i(j-1) before PV_i(j-1) has read it, and a tcgen05.commit
+// tracks every MMA the thread issued before it: when softmax i sees S_i(j)
+// complete, PV_i(j-1) is complete too and O_i may be rescaled in place.  K and
+// V stages are freed by count-2 mbarriers with one commit after each of the two
+// MMAs reading the stage.  The tensor core runs PV1(j-1), S1(j) while softmax 0
+// works on S0(j), and PV0(j), S0(j+1) while softmax 1 works on S1(j); the two
+// softmax warpgroups take turns on the ex2 unit.  Thread-to-thread hand-offs
+// (P ready -> MMA warp, the ping-pong turns) use named barriers, which are
+// far cheaper than an mbarrier round trip; mbarriers remain only where the
+// tensor core or the TMA unit signals.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -56,7 +57,7 @@ struct AttnCfg {
   static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
   static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
   static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2;
   static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 16;
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
@@ -106,10 +107,11 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* k_empty = k_full + NK;
   uint64_t* v_full = k_empty + NK;
   uint64_t* v_empty = v_full + NV;
-  uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed
-  uint64_t* p_ready = s_full + 2;    // [2] softmax i finished tile j (128 arrivals)
-  uint64_t* pv_done = p_ready + 2;   // [2] PV_i(j) computed
-  uint64_t* turn = pv_done + 2;      // [2] softmax i may exponentiate (ping-pong between the warpgroups)
+  uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and every earlier MMA)
+  uint64_t* pv_done = s_full + 2;    // [2] PV_i(j) computed (read by the epilogue)
+  // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
+  //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
+  constexpr uint32_t kBarPReady = 1, kBarTurn = 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
 
   const int warp = threadIdx.x >> 5;
@@ -123,9 +125,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(s_full + i, 1);
-      mbar_init(p_ready + i, 128);
       mbar_init(pv_done + i, 1);
-      mbar_init(turn + i, 128);
     }
     for (int s = 0; s < NK; ++s) {
       mbar_init(k_full + s, 1);
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the schedule (named barriers are warp-aligned); lane 0 issues.
       constexpr uint32_t fmt = FP8 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
       constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, BM, BN);  // Q, K both K-major
       constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 1, BM, D);   // V MN-major (d contiguous)
@@ -210,47 +210,60 @@ __global__ void __launch_bounds__(384, 1)
             mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      const bool leader = lane == 0;
       bool ok = mbar_wait(q_full, 0, err, kErrTimeout) && mbar_wait(k_full, 0, err, kErrTimeout);
+      ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        qk(0, 0);
-        mma_commit(s_full);
-        mma_commit(k_empty);
-        ok = mbar_wait(q_full + 1, 0, err, kErrTimeout);
+        if (leader) {
+          qk(0, 0);
+          mma_commit(s_full);
+          mma_commit(k_empty);
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(q_full + 1, 0, err, kErrTimeout));
       }
       if (ok) {
         tc_fence_after();
-        qk(1, 0);
-        mma_commit(s_full + 1);
-        mma_commit(k_empty);
+        if (leader) {
+          qk(1, 0);
+          mma_commit(s_full + 1);
+          mma_commit(k_empty);
+        }
       }
+      __syncwarp();
       for (int j = 1; ok && j <= nkv; ++j) {
         const int jj = j - 1, sv = jj % NV, sk = j % NK;
-        if (!mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout)) break;
-        if (!mbar_wait(p_ready, jj & 1, err, kErrTimeout)) break;
+        // TMA readiness first, while the softmax warpgroups are still busy
+        ok = mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout);
+        if (ok && j < nkv) ok = mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        named_sync<kBarPReady + 0, 160>();
         tc_fence_after();
-        pv(0, sv, jj > 0);
-        mma_commit(pv_done);
-        mma_commit(v_empty + sv);
-        if (j < nkv) {
-          if (!mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout)) break;
-          tc_fence_after();
-          qk(0, sk);
-          mma_commit(s_full);
-          mma_commit(k_empty + sk);
+        if (leader) {
+          pv(0, sv, jj > 0);
+          mma_commit(pv_done);
+          mma_commit(v_empty + sv);
+          if (j < nkv) {
+            qk(0, sk);
+            mma_commit(s_full);
+            mma_commit(k_empty + sk);
+          }
         }
-        if (!mbar_wait(p_ready + 1, jj & 1, err, kErrTimeout)) break;
+        __syncwarp();
+        named_sync<kBarPReady + 1, 160>();
         tc_fence_after();
-        pv(1, sv, jj > 0);
-        mma_commit(pv_done + 1);
-        mma_commit(v_empty + sv);
-        if (j < nkv) {
-          qk(1, sk);
-          mma_commit(s_full + 1);
-          mma_commit(k_empty + sk);
+        if (leader) {
+          pv(1, sv, jj > 0);
+          mma_commit(pv_done + 1);
+          mma_commit(v_empty + sv);
+          if (j < nkv) {
+            qk(1, sk);
+            mma_commit(s_full + 1);
+            mma_commit(k_empty + sk);
+          }
         }
+        __syncwarp();
       }
-    }
    }
   } else {
     regs_inc<C::kRegsSoftmax>();
@@ -283,8 +296,6 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, j & 1, err, kErrTimeout));
-      // PV_i(j-1) done: O_i may be rescaled (consumed every tile, so phases stay in step)
-      if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, (j - 1) & 1, err, kErrTimeout));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[BN];
@@ -327,10 +338,8 @@ __global__ void __launch_bounds__(384, 1)
       // Ping-pong: the two warpgroups take turns on the ex2 unit, so one exponentiates
       // while the other's PV and next S run on the tensor core.  Softmax 0 goes first in
       // every tile; softmax 1 starts tile j once softmax 0 has finished tile j's exps.
-      if (i == 1 || j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(turn + i, (i == 1 ? j : j - 1) & 1, err, kErrTimeout));
-        if (!ok) break;
-      }
+      if (i == 1) named_sync<kBarTurn + 1, 256>();
+      else if (j > 0) named_sync<kBarTurn + 0, 256>();
       // p = 2^(s * c - m): packed scale-and-subtract, ex2 per element, packed row
       // sums in 4 chains (in the shadow of the ex2 pipe), P to TMEM per 32 keys.
       // tcgen05.st reads its source registers asynchronously: every register a
@@ -373,10 +382,12 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st16(tS + 16 * q, p + 16 * q);
         }
       }
-      mbar_arrive(turn + (i ^ 1));
+      // every arrive is matched by a sync of the other warpgroup
+      if (i == 0) named_arrive<kBarTurn + 1, 256>();
+      else if (j + 1 < nkv) named_arrive<kBarTurn + 0, 256>();
       tmem_wait_st();
       reg_fence(p);
-      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1) (pv_done waited above)
+      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1): the commit behind S_i(j) covers them
         uint32_t o[D];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o + c * 32);
@@ -396,7 +407,8 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(o);
       }
       tc_fence_before();
-      mbar_arrive(p_ready + i);
+      if (i == 0) named_arrive<kBarPReady + 0, 160>();
+      else named_arrive<kBarPReady + 1, 160>();
       float a0, a1;
       f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
       l = l * alpha + (a0 + a1);

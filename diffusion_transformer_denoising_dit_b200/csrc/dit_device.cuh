@@ -261,6 +261,17 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt
          ((M >> 4) << 24);
 }
 
+// Named CTA barriers (ids 1..15; 0 is __syncthreads).  `count` threads take part
+// in each generation: arrivers do not wait, syncers wait for the generation.
+template <uint32_t ID, uint32_t COUNT>
+__device__ __forceinline__ void named_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(COUNT) : "memory");
+}
+template <uint32_t ID, uint32_t COUNT>
+__device__ __forceinline__ void named_arrive() {
+  asm volatile("bar.arrive %0, %1;" ::"n"(ID), "n"(COUNT) : "memory");
+}
+
 // Warpgroup register re-split (all four warps of a warpgroup execute the same one).
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {
