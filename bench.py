@@ -262,9 +262,9 @@ def run_ours(args, rank, world, local_rank):
     ms_attn = timed(lambda: dit.attention(qr, kr, v, out=o), ka, 3) / ka
     achieved = flops / (ms_attn / 1e3) / 1e12
     bf16_peak = peaks["bf16_tflops"]
-    h_attn = _src_hash("attn_bf16.cu", "dit_device.cuh")
+    h_attn = _src_hash("attn_kernel.cuh", "dit_device.cuh", "attn_bf16.cu")
     tr = NCU_TRAFFIC.get(("attn_bf16", h_attn))
-    roofline = {"bound": "tensor", "kernel": "attn_bf16_kernel<128>", "achieved": achieved, "peak": bf16_peak,
+    roofline = {"bound": "tensor", "kernel": "attn_kernel<bf16, d=128>", "achieved": achieved, "peak": bf16_peak,
                 "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": tr,
                 "peak_source": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
                 "frac_of_nominal_2250": achieved / 2250.0, "ms_per_launch": ms_attn}
@@ -356,6 +356,84 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------- denoising trace
+def run_trace(args):
+    """28-step denoising trace at 2048 px: per step, block 0's attention runs, the
+    First-Block-Cache gate compares its residual with the previous step's, and
+    unless the gate says skip the remaining 56 attention calls of the step run
+    (19 joint + 38 single blocks = 57 calls per computed step).  The same call
+    sequence is run once with the gate and once without it; both are timed on
+    the device.  Q/K/V rotate over 4 seeded sets so that no call reuses L2."""
+    import torch
+    import diffusion_transformer_denoising_dit_b200 as dit
+    from diffusion_transformer_denoising_dit_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[WORKLOAD]
+    steps, blocks, thr = 28, 57, THRESHOLD
+    sets = [synth.qkv(w, device=dev, seed=w.seed + 100 + i) for i in range(4)]
+    pos = synth.positions(w.T, w.G).to(dev)
+    cos, sin = dit.rope_tables(pos, w.axes, w.theta)
+    o = torch.empty_like(sets[0][0])
+    ws = dit.attention_workspace(w.B, w.H, w.N, w.d, "bf16", rope=True, device=dev)
+    res = list(synth.drift_residuals(w.N, HIDDEN, steps=steps, device=dev))
+    gate = dit.FBCacheGate(thr, res[0].numel(), device=dev)
+    expected = [False] + [d < thr for d in synth.drift_schedule(steps)]
+    rel_seen = []
+
+    def attn(c):
+        q, k, v = sets[c % 4]
+        dit.attention(q, k, v, cos, sin, out=o, workspace=ws)
+
+    def run(use_gate):
+        calls, skipped = 0, []
+        per_step = []
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for t in range(steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn(calls)
+            calls += 1
+            skip = False
+            if use_gate and t > 0:
+                flag = gate(res[t], res[t - 1])
+                skip = bool(flag.item())        # the step's one device-to-host read
+                rel_seen.append(float(gate.rel.item()))
+            if not skip:
+                for _ in range(blocks - 1):
+                    attn(calls)
+                    calls += 1
+            else:
+                skipped.append(t)
+            e1.record()
+            per_step.append((e0, e1))
+        t1 = torch.cuda.Event(enable_timing=True)
+        t1.record()
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1), calls, skipped, [a.elapsed_time(b) for a, b in per_step]
+
+    for _ in range(3):
+        attn(0)
+    base_ms, base_calls, _, base_steps = run(False)
+    gated_ms, gated_calls, skipped, gated_steps = run(True)
+    assert dit.read_error() == 0
+    line = {
+        "metric": "28-step 2048px denoising attention trace with First-Block-Cache (threshold %.2f)" % thr,
+        "unit": "ms", "higher_is_better": False, "data": "synthetic",
+        "config": {"workload": "flux2k attention x (19 joint + 38 single) blocks x 28 steps; residuals "
+                               "16896x3072 bf16 with seeded geometric drift 0.4 -> 0.02"},
+        "no_skip": {"ms": base_ms, "attention_calls": base_calls, "ms_per_computed_step": sum(base_steps) / steps},
+        "fbcache": {"ms": gated_ms, "attention_calls": gated_calls, "skipped_steps": skipped,
+                    "skipped_expected_from_drift": [t for t, s in enumerate(expected) if s],
+                    "rel_per_step": rel_seen},
+        "speedup": base_ms / gated_ms,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -364,6 +442,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="run the 28-step denoising trace instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -372,6 +451,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.trace:
+        run_trace(args)
         return
     if world > 1:
         import datetime
