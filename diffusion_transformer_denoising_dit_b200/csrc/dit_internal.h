@@ -67,7 +67,7 @@ struct Fp8Prep {
   float* k_partial;    // [B*H][kFp8MeanChunks][128] K-mean partial sums
 };
 
-constexpr int kFp8MeanChunks = 16;
+constexpr int kFp8MeanChunks = 48;
 
 cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream);
 

@@ -9,12 +9,12 @@
 // channel mean over all N tokens after rotation (which leaves softmax
 // unchanged in exact arithmetic).
 //
-// Pass 1 (kmean_partial): per (b,h) and token chunk, fp32 channel sums of the
+// Pass 1 (kmean_partial): per (b,h) and one of 48 token chunks, fp32 channel sums of the
 //   rotated K; also clears the per-(b,h) V scale maximum.
-// Pass 2 (quantize): one CTA per (b,h, 128-token block): rotate Q and K in
-//   fp32, subtract the K mean (partials combined in a fixed order), block
-//   amax, scale and cast to e4m3; write the scales.  Streams 6 B/element in
-//   (bf16 Q, K, V) and 3 B/element out; HBM-bound.
+// Pass 2 (quantize): one CTA per (128-token block, (b,h), tensor): rotate Q
+//   and K in fp32, subtract the K mean (partials combined in a fixed order),
+//   block amax, scale and cast to e4m3; write the scales.  Streams 6 B/element
+//   in (bf16 Q, K, V) and 3 B/element out; HBM-bound.
 #include <cuda_bf16.h>
 
 #include "dit_device.cuh"
@@ -142,9 +142,14 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
   }
 }
 
-__global__ void __launch_bounds__(kThreads) quantize_qkv(Fp8Prep p, const float* __restrict__ partial) {
+// One CTA per (128-token block, (b,h), tensor): blockIdx.z = 0 quantises Q (one
+// 128-token block, rotated), 1 quantises K (two 64-token blocks, rotated and
+// smoothed), 2 quantises V (two 64-token blocks).  Every thread issues its eight
+// 16-byte loads before any reduction, so each CTA keeps 32 KB in flight.
+__global__ void __launch_bounds__(kThreads, 2) quantize_qkv(Fp8Prep p, const float* __restrict__ partial) {
   const int blk = blockIdx.x;  // 128-token block
   const int bh = blockIdx.y;
+  const int which = blockIdx.z;
   const int b = bh / p.H, h = bh % p.H;
   const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
   const int n_base = blk * 128;
@@ -152,67 +157,63 @@ __global__ void __launch_bounds__(kThreads) quantize_qkv(Fp8Prep p, const float*
   __shared__ float mean[128];
   __shared__ float red[16];
   __shared__ float unused_scale;  // sink for the second scale of a block past the sequence end
-  if (threadIdx.x < 128) {
-    float s = 0.f;
-    if (p.smooth_k)
-      for (int c = 0; c < kChunks; ++c) s += partial[(static_cast<int64_t>(bh) * kChunks + c) * 128 + threadIdx.x];
-    const float m = s / static_cast<float>(p.N);
-    mean[threadIdx.x] = m;
-    if (blk == 0) p.k_mean[bh * 128 + threadIdx.x] = m;
-  }
-  __syncthreads();
   const int64_t out_off = static_cast<int64_t>(bh) * p.N * 128;
-  float x[8][8];
-  // ---- Q: one 128-token block
-  {
-    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.q) + b * p.sq[0] + h * p.sq[1];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int n = n_base + tl + 16 * i;
-      if (n < p.N)
-        load_rotate8(src + static_cast<int64_t>(n) * p.sq[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, 64, x[i]);
-      else
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
-    }
-    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr);
+  const __nv_bfloat16* src;
+  int64_t tok_stride;
+  const float* ct = nullptr;
+  const float* st = nullptr;
+  if (which == 0) {
+    src = static_cast<const __nv_bfloat16*>(p.q) + b * p.sq[0] + h * p.sq[1];
+    tok_stride = p.sq[2];
+    ct = p.cos_tab;
+    st = p.sin_tab;
+  } else if (which == 1) {
+    src = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
+    tok_stride = p.sk[2];
+    ct = p.cos_tab;
+    st = p.sin_tab;
+  } else {
+    src = static_cast<const __nv_bfloat16*>(p.v) + b * p.sv[0] + h * p.sv[1];
+    tok_stride = p.sv[2];
   }
-  // ---- K: two 64-token blocks, smoothed
-  {
-    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
+  float x[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = n_base + tl + 16 * i;
+    if (n < p.N)
+      load_rotate8(src + static_cast<int64_t>(n) * tok_stride + cc * 8, ct, st, n, cc, 64, x[i]);
+    else
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+  }
+  if (which == 0) {
+    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr);
+    return;
+  }
+  if (which == 1) {
+    if (threadIdx.x < 128) {
+      float sum = 0.f;
+      if (p.smooth_k)
+        for (int c = 0; c < kChunks; ++c) sum += partial[(static_cast<int64_t>(bh) * kChunks + c) * 128 + threadIdx.x];
+      const float m = sum / static_cast<float>(p.N);
+      mean[threadIdx.x] = m;
+      if (blk == 0) p.k_mean[bh * 128 + threadIdx.x] = m;
+    }
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int n = n_base + tl + 16 * i;
-      if (n < p.N) {
-        load_rotate8(src + static_cast<int64_t>(n) * p.sk[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, 64, x[i]);
+      if (n_base + tl + 16 * i < p.N) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[i][e] -= mean[cc * 8 + e];
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
       }
     }
     float* s1 = (2 * blk + 1 < nk) ? p.k_scale + bh * nk + 2 * blk + 1 : &unused_scale;
     quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr);
+    return;
   }
-  // ---- V: two 64-token blocks, no rotation
-  {
-    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.v) + b * p.sv[0] + h * p.sv[1];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int n = n_base + tl + 16 * i;
-      if (n < p.N)
-        load_rotate8(src + static_cast<int64_t>(n) * p.sv[2] + cc * 8, nullptr, nullptr, n, cc, 64, x[i]);
-      else
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
-    }
-    const bool has2 = 2 * blk + 1 < nk;
-    float* s1 = has2 ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
-    quantize_tile(x, true, n_base, p.N, p.v8 + out_off, cc, tl, red, p.v_scale + bh * nk + 2 * blk, s1,
-                  p.v_scale_max + bh);
-  }
-  (void)nq;
+  float* s1 = (2 * blk + 1 < nk) ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
+  quantize_tile(x, true, n_base, p.N, p.v8 + out_off, cc, tl, red, p.v_scale + bh * nk + 2 * blk, s1,
+                p.v_scale_max + bh);
 }
 
 }  // namespace
@@ -223,7 +224,7 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
   kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 g2((p.N + 127) / 128, p.B * p.H);
+  dim3 g2((p.N + 127) / 128, p.B * p.H, 3);
   quantize_qkv<<<g2, kThreads, 0, stream>>>(p, partial);
   return cudaGetLastError();
 }

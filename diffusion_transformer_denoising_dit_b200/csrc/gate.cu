@@ -9,7 +9,7 @@
 // Cache-DiT on the TensorRT-LLM VisualGen page).
 //
 // HBM-bound: 4 bytes read per element, ~3 flops.  Pass 1 streams both inputs
-// with 16-byte loads over a grid of (SMs x 8) CTAs, fp32 per-thread partials,
+// with 16-byte loads (4 per input in flight per thread) over up to 1184 CTAs, fp32 per-thread partials,
 // fp64 per-CTA combine; pass 2 (one CTA) combines the CTA partials in a fixed
 // tree order, so the result is deterministic for a given n.
 #include <cuda_bf16.h>
@@ -53,14 +53,18 @@ __global__ void __launch_bounds__(kGateThreads) gate_pass1(const __nv_bfloat16* 
   const uint4* b8 = reinterpret_cast<const uint4*>(b);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  // two independent 16-byte loads of each input in flight per iteration
-  for (; i + stride < n8; i += 2 * stride) {
-    const uint4 av0 = __ldcs(a8 + i), bv0 = __ldcs(b8 + i);
-    const uint4 av1 = __ldcs(a8 + i + stride), bv1 = __ldcs(b8 + i + stride);
-    accum8(av0, bv0, num, den);
-    accum8(av1, bv1, num, den);
+  // four independent 16-byte loads of each input in flight per iteration
+  for (; i + 3 * stride < n8; i += 4 * stride) {
+    uint4 av[4], bv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      av[u] = __ldcs(a8 + i + u * stride);
+      bv[u] = __ldcs(b8 + i + u * stride);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) accum8(av[u], bv[u], num, den);
   }
-  if (i < n8) accum8(__ldcs(a8 + i), __ldcs(b8 + i), num, den);
+  for (; i < n8; i += stride) accum8(__ldcs(a8 + i), __ldcs(b8 + i), num, den);
   if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {  // ragged tail (< 8 elements)
     const int64_t t = n8 * 8 + threadIdx.x;
     const float x = __bfloat162float(a[t]);
