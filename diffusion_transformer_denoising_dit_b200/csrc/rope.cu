@@ -57,7 +57,13 @@ struct RopeArgs {
 // Consecutive threads walk consecutive 16-byte chunks of a token row; each
 // thread handles kUnroll chunks a grid-stride apart and issues all their loads
 // before any arithmetic, so enough bytes are in flight to saturate HBM.
-constexpr int kUnroll = 4;
+#ifndef DIT_ROPE_UNROLL
+#define DIT_ROPE_UNROLL 1
+#endif
+#ifndef DIT_ROPE_CTAS_PER_SM
+#define DIT_ROPE_CTAS_PER_SM 0
+#endif
+constexpr int kUnroll = DIT_ROPE_UNROLL;
 
 __device__ __forceinline__ void rope_chunk(const RopeArgs& a, const RopeJob& jb, int64_t idx, int cpr, uint4& xv,
                                            float4& cv, float4& sv, int64_t& yo) {
@@ -74,7 +80,7 @@ __device__ __forceinline__ void rope_chunk(const RopeArgs& a, const RopeJob& jb,
   sv = *reinterpret_cast<const float4*>(a.sin_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
 }
 
-__global__ void __launch_bounds__(256, 4) rope_apply_kernel(RopeArgs a) {
+__global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
   const RopeJob& jb = a.job[blockIdx.y];
   const int cpr = a.d / 8;  // chunks per row
   const int64_t total = static_cast<int64_t>(a.B) * a.H * a.N * cpr;
@@ -130,8 +136,10 @@ cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int 
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int64_t blocks = (total + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(sms) * 4;  // 4 resident 256-thread CTAs per SM
-  if (blocks > cap) blocks = cap;
+  if (DIT_ROPE_CTAS_PER_SM > 0) {  // optional persistent-style cap (grid-stride loop)
+    const int64_t cap = static_cast<int64_t>(sms) * DIT_ROPE_CTAS_PER_SM;
+    if (blocks > cap) blocks = cap;
+  }
   dim3 grid(static_cast<unsigned>(blocks), njobs);
   rope_apply_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
