@@ -45,7 +45,7 @@ namespace dit {
 template <bool FP8, int D>
 struct AttnCfg {
   static constexpr int BM = 128;                        // rows per Q tile (two per CTA)
-  static constexpr int BN = 128;                        // keys per K/V tile
+  static constexpr int BN = kAttnBlockN;                // keys per K/V tile (128)
   static constexpr int kThreads = 384;
   static constexpr uint32_t kRegsSoftmax = 208, kRegsAux = 80;
   static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= 65536, "register re-split exceeds the register file");

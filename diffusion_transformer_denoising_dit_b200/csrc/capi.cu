@@ -203,9 +203,10 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
     for (int i = 0; i < 3; ++i) sqa[i] = ska[i] = cs[i];
   }
   CUtensorMap tq, tk, tv;
+  // Q tiles are 128 tokens, K/V tiles kAttnBlockN tokens; boxes are 128 bytes wide.
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qa, B, H, N, d, sqa, 64, 128) ||
-      !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ka, B, H, N, d, ska, 64, 128) ||
-      !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, B, H, N, d, sv, 64, 128))
+      !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ka, B, H, N, d, ska, 64, dit::kAttnBlockN) ||
+      !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, B, H, N, d, sv, 64, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
   dit::AttnOut out;
   out.o = o;
@@ -270,8 +271,8 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   CUtensorMap tq, tk, tv;
   // e4m3: one 128-byte row holds all d = 128 channels of a token.
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.q8, B, H, N, d, cs, 128, 128) ||
-      !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.k8, B, H, N, d, cs, 128, 128) ||
-      !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.v8, B, H, N, d, cs, 128, 128))
+      !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.k8, B, H, N, d, cs, 128, dit::kAttnBlockN) ||
+      !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.v8, B, H, N, d, cs, 128, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
   dit::AttnOut out;
   out.o = o;

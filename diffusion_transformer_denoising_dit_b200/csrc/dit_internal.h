@@ -8,6 +8,9 @@
 
 namespace dit {
 
+// Keys per K/V tile of the attention kernels (the TMA box height of the K and V maps).
+constexpr int kAttnBlockN = 128;
+
 // Error codes written to the device error word (match dit_status).
 constexpr int kErrTimeout = 6;
 

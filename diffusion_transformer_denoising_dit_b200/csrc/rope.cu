@@ -54,19 +54,15 @@ struct RopeArgs {
 
 // One thread per 8 consecutive channels (4 pairs): one 16-byte load of x, two
 // 16-byte loads of the tables, one 16-byte (bf16) or two (fp32) stores.
-// Consecutive threads walk consecutive 16-byte chunks of a token row; each
-// thread handles kUnroll chunks a grid-stride apart and issues all their loads
-// before any arithmetic, so enough bytes are in flight to saturate HBM.
-#ifndef DIT_ROPE_UNROLL
-#define DIT_ROPE_UNROLL 1
-#endif
-#ifndef DIT_ROPE_CTAS_PER_SM
-#define DIT_ROPE_CTAS_PER_SM 0
-#endif
-constexpr int kUnroll = DIT_ROPE_UNROLL;
-
-__device__ __forceinline__ void rope_chunk(const RopeArgs& a, const RopeJob& jb, int64_t idx, int cpr, uint4& xv,
-                                           float4& cv, float4& sv, int64_t& yo) {
+// Consecutive threads walk consecutive 16-byte chunks of a token row; the grid
+// covers every chunk once (measured faster than a grid-stride loop or several
+// chunks per thread, which cost occupancy).
+__global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
+  const RopeJob& jb = a.job[blockIdx.y];
+  const int cpr = a.d / 8;  // chunks per row
+  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.N * cpr;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
   const int c = static_cast<int>(idx % cpr);
   const int64_t row = idx / cpr;
   const int n = static_cast<int>(row % a.N);
@@ -74,53 +70,31 @@ __device__ __forceinline__ void rope_chunk(const RopeArgs& a, const RopeJob& jb,
   const int h = static_cast<int>(bh % a.H);
   const int b = static_cast<int>(bh / a.H);
   const int64_t xo = b * jb.sx[0] + h * jb.sx[1] + n * jb.sx[2] + c * 8;
-  yo = b * jb.sy[0] + h * jb.sy[1] + n * jb.sy[2] + c * 8;
-  xv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(jb.x) + xo);
-  cv = *reinterpret_cast<const float4*>(a.cos_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
-  sv = *reinterpret_cast<const float4*>(a.sin_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
-}
-
-__global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
-  const RopeJob& jb = a.job[blockIdx.y];
-  const int cpr = a.d / 8;  // chunks per row
-  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.N * cpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
-       base += kUnroll * stride) {
-    uint4 xv[kUnroll];
-    float4 cv[kUnroll], sv[kUnroll];
-    int64_t yo[kUnroll];
+  const int64_t yo = b * jb.sy[0] + h * jb.sy[1] + n * jb.sy[2] + c * 8;
+  const uint4 xv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(jb.x) + xo);
+  const float4 cv = *reinterpret_cast<const float4*>(a.cos_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
+  const float4 sv = *reinterpret_cast<const float4*>(a.sin_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
+  const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
+  const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+  const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+  float y[8];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t idx = base + u * stride;
-      if (idx < total) rope_chunk(a, jb, idx, cpr, xv[u], cv[u], sv[u], yo[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (base + u * stride >= total) break;
-      const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv[u]);
-      const float cc[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
-      const float ss[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
-      float y[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x2 = __bfloat1622float2(xp[i]);
-        y[2 * i] = x2.x * cc[i] - x2.y * ss[i];
-        y[2 * i + 1] = x2.x * ss[i] + x2.y * cc[i];
-      }
-      if (a.out_fp32) {
-        float4* yp = reinterpret_cast<float4*>(static_cast<float*>(jb.y) + yo[u]);
-        yp[0] = make_float4(y[0], y[1], y[2], y[3]);
-        yp[1] = make_float4(y[4], y[5], y[6], y[7]);
-      } else {
-        uint4 o;
-        o.x = pack_bf16x2(y[0], y[1]);
-        o.y = pack_bf16x2(y[2], y[3]);
-        o.z = pack_bf16x2(y[4], y[5]);
-        o.w = pack_bf16x2(y[6], y[7]);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(jb.y) + yo[u]) = o;
-      }
-    }
+  for (int i = 0; i < 4; ++i) {
+    const float2 x2 = __bfloat1622float2(xp[i]);
+    y[2 * i] = x2.x * cc[i] - x2.y * ss[i];
+    y[2 * i + 1] = x2.x * ss[i] + x2.y * cc[i];
+  }
+  if (a.out_fp32) {
+    float4* yp = reinterpret_cast<float4*>(static_cast<float*>(jb.y) + yo);
+    yp[0] = make_float4(y[0], y[1], y[2], y[3]);
+    yp[1] = make_float4(y[4], y[5], y[6], y[7]);
+  } else {
+    uint4 o;
+    o.x = pack_bf16x2(y[0], y[1]);
+    o.y = pack_bf16x2(y[2], y[3]);
+    o.z = pack_bf16x2(y[4], y[5]);
+    o.w = pack_bf16x2(y[6], y[7]);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(jb.y) + yo) = o;
   }
 }
 
@@ -132,14 +106,7 @@ cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int 
   a.B = B; a.H = H; a.N = N; a.d = d;
   a.cos_tab = cos_tab; a.sin_tab = sin_tab; a.out_fp32 = out_fp32;
   const int64_t total = static_cast<int64_t>(B) * H * N * (d / 8);
-  int sms = 148;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = (total + 255) / 256;
-  if (DIT_ROPE_CTAS_PER_SM > 0) {  // optional persistent-style cap (grid-stride loop)
-    const int64_t cap = static_cast<int64_t>(sms) * DIT_ROPE_CTAS_PER_SM;
-    if (blocks > cap) blocks = cap;
-  }
+  const int64_t blocks = (total + 255) / 256;
   dim3 grid(static_cast<unsigned>(blocks), njobs);
   rope_apply_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
