@@ -62,9 +62,16 @@ struct AttnCfg {
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
   static constexpr uint32_t kTmemCols = 512;
-  // lazy rescale threshold (log2 units): with a stale max every p <= 2^kRescaleLog2.
-  // e4m3 P (p * 448 * sV / sV_max) has no headroom for that, so FP8 rescales on any growth.
-  static constexpr float kRescaleLog2 = FP8 ? 0.f : 8.f;
+  // Lazy rescale threshold tau (log2 units): O and l stay in the frame of a stale
+  // max m until a row's tile max exceeds m + tau, so every p = 2^(x - m) <= 2^tau.
+  // BF16: tau = 8 (a larger tau keeps the range but rounds the dominant p of a
+  // near-one-hot row to bf16 in a stale frame, which costs accuracy).  FP8: e4m3 P is
+  // stored as p * 2^-tau * 448 * sV / sV_max <= 448, so tau buys fewer rescales
+  // at the price of smaller P codes; at tau = 4 only p < 2^-11 (relative to the
+  // row max) falls below the e4m3 normal range.
+  static constexpr int kTau = FP8 ? 4 : 8;
+  static constexpr float kRescaleLog2 = static_cast<float>(kTau);
+  static constexpr float kTwoTau = static_cast<float>(1ull << kTau);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kRowBytes % 128 == 0, "token rows must be whole 128-byte swizzle atoms");
 };
@@ -83,6 +90,12 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
@@ -275,7 +288,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + C::kColO + D * i + lane_off;
     const float sl2 = out.scale_log2;
     const int qblk = 2 * qt + i;                // 128-row block index of this Q tile
-    // FP8 scales: score = S * sQ * sK(j) * scale, P8 = p * 448 * sV(j) / sV_max
+    // FP8 scales: score = S * sQ * sK(j) * scale, P8 = p * 2^-tau * 448 * sV(j) / sV_max
     float qs = sl2, vfold = 1.f, fin_scale = 1.f;
     const float* ksc = nullptr;
     const float* vsc = nullptr;
@@ -288,8 +301,8 @@ __global__ void __launch_bounds__(384, 1)
       vsc = sc.v_scale + static_cast<int64_t>(bh) * nk;
       const float vmax = sc.v_scale_max[bh];
       qs = (qblk < nq ? sc.q_scale[static_cast<int64_t>(bh) * nq + qblk] : 1.f) * sl2;
-      vfold = 448.f / vmax;
-      fin_scale = vmax / 448.f;
+      vfold = 448.f / (vmax * C::kTwoTau);
+      fin_scale = vmax * C::kTwoTau / 448.f;
     }
     float m = -INFINITY;  // running (possibly stale) max of the scaled log2 scores
     float l = 0.f;
@@ -316,7 +329,7 @@ __global__ void __launch_bounds__(384, 1)
         c0 = qs * ksc[kb0];
         c1 = kb1 < nk ? qs * ksc[kb1] : 1.f;  // past the end every key is -inf; keep -inf * c1 = -inf
         f0 = vsc[kb0] * vfold;
-        f1 = kb1 < nk ? vsc[kb1] * vfold : 0.f;
+        f1 = kb1 < nk ? vsc[kb1] * vfold : 1.f;  // past the end every p is 0 anyway
       }
       // row max: two 3-input max chains per 64-key half
       float ma0 = __uint_as_float(s[0]), ma1 = __uint_as_float(s[1]);
@@ -346,6 +359,10 @@ __global__ void __launch_bounds__(384, 1)
       // pending store reads stays pinned (reg_fence after tcgen05.wait::st) so the
       // compiler cannot reuse it before the store has completed.
       const uint64_t nm2 = f2(-m_new, -m_new);
+      // FP8: the V block scale of each 64-key half enters as an exponent offset,
+      // p * f = 2^(x - m + log2 f), which saves a multiply per element.
+      const float lf0 = FP8 ? lg2(f0) - m_new : 0.f, lf1 = FP8 ? lg2(f1) - m_new : 0.f;
+      const uint64_t nmA = f2(lf0, lf0), nmB = f2(lf1, lf1);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       constexpr int kPRegs = FP8 ? 32 : 64;  // packed P of the whole row
       uint32_t p[kPRegs];
@@ -353,19 +370,17 @@ __global__ void __launch_bounds__(384, 1)
       for (int q = 0; q < 4; ++q) {  // 32 keys per TMEM store
         const uint64_t cq = FP8 ? (q < 2 ? f2(c0, c0) : f2(c1, c1)) : f2(sl2, sl2);
         if constexpr (FP8) {  // 32 keys -> 8 columns of 4 e4m3 (V block scale folded in)
-          const uint64_t fv = q < 2 ? f2(f0, f0) : f2(f1, f1);
+          const uint64_t nmq = q < 2 ? nmA : nmB;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int k0 = 32 * q + 4 * e;
             float x0, x1, x2, x3;
-            f2_split(ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), cq, nm2), x0, x1);
-            f2_split(ffma2(f2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), cq, nm2), x2, x3);
-            const uint64_t pa = f2(ex2(x0), ex2(x1)), pb = f2(ex2(x2), ex2(x3));
-            acc[(2 * e) & 3] = fadd2(acc[(2 * e) & 3], pa);
-            acc[(2 * e + 1) & 3] = fadd2(acc[(2 * e + 1) & 3], pb);
-            float a, bq, cc, dd;
-            f2_split(fmul2(pa, fv), a, bq);
-            f2_split(fmul2(pb, fv), cc, dd);
+            f2_split(ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), cq, nmq), x0, x1);
+            f2_split(ffma2(f2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), cq, nmq), x2, x3);
+            const float a = ex2(x0), bq = ex2(x1), cc = ex2(x2), dd = ex2(x3);
+            // row sums per 64-key half (each carries its own V block scale)
+            acc[2 * (q >> 1)] = fadd2(acc[2 * (q >> 1)], f2(a, bq));
+            acc[2 * (q >> 1) + 1] = fadd2(acc[2 * (q >> 1) + 1], f2(cc, dd));
             p[8 * q + e] = cvt_e4m3x4(a, bq, cc, dd);
           }
           tmem_st8(tS + 8 * q, p + 8 * q);
@@ -410,8 +425,15 @@ __global__ void __launch_bounds__(384, 1)
       if (i == 0) named_arrive<kBarPReady + 0, 160>();
       else named_arrive<kBarPReady + 1, 160>();
       float a0, a1;
-      f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
-      l = l * alpha + (a0 + a1);
+      if constexpr (FP8) {  // divide each half's V block scale back out of its row sum
+        float b0, b1;
+        f2_split(fadd2(acc[0], acc[1]), a0, a1);
+        f2_split(fadd2(acc[2], acc[3]), b0, b1);
+        l = l * alpha + ((a0 + a1) * __frcp_rn(f0) + (b0 + b1) * __frcp_rn(f1));
+      } else {
+        f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+        l = l * alpha + (a0 + a1);
+      }
       m = m_new;
     }
     // ---------------------------------------------------------- epilogue

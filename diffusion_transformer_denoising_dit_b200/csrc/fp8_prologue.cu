@@ -11,8 +11,9 @@
 //
 // Pass 1 (kmean_partial): per (b,h) and one of 48 token chunks, fp32 channel sums of the
 //   rotated K; also clears the per-(b,h) V scale maximum.
+// Pass 1b (kmean_finalize): the partials of each (b,h) combined in a fixed order.
 // Pass 2 (quantize): one CTA per (128-token block, (b,h), tensor): rotate Q
-//   and K in fp32, subtract the K mean (partials combined in a fixed order),
+//   and K in fp32, subtract the K mean,
 //   block amax, scale and cast to e4m3; write the scales.  Streams 6 B/element
 //   in (bf16 Q, K, V) and 3 B/element out; HBM-bound.
 #include <cuda_bf16.h>
@@ -100,6 +101,20 @@ __global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __re
   }
 }
 
+// K channel means: one CTA per (b,h), thread c sums the kChunks partials of
+// channel c in a fixed order (independent loads, then the adds).
+__global__ void __launch_bounds__(128) kmean_finalize(Fp8Prep p, const float* __restrict__ partial) {
+  const int bh = blockIdx.x;
+  const int c = threadIdx.x;
+  float v[kChunks];
+#pragma unroll
+  for (int k = 0; k < kChunks; ++k) v[k] = partial[(static_cast<int64_t>(bh) * kChunks + k) * 128 + c];
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kChunks; ++k) sum += v[k];
+  p.k_mean[bh * 128 + c] = p.smooth_k ? sum / static_cast<float>(p.N) : 0.f;
+}
+
 // Quantises one 128-token block of one tensor held as 8 chunks per thread:
 // thread t owns channel chunk (t % 16) of tokens t/16 + 16 i, i = 0..7.  With
 // two_blocks the first four tokens of a thread lie in the first 64-token block.
@@ -146,7 +161,7 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
 // 128-token block, rotated), 1 quantises K (two 64-token blocks, rotated and
 // smoothed), 2 quantises V (two 64-token blocks).  Every thread issues its eight
 // 16-byte loads before any reduction, so each CTA keeps 32 KB in flight.
-__global__ void __launch_bounds__(kThreads, 2) quantize_qkv(Fp8Prep p, const float* __restrict__ partial) {
+__global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
   const int blk = blockIdx.x;  // 128-token block
   const int bh = blockIdx.y;
   const int which = blockIdx.z;
@@ -191,14 +206,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_qkv(Fp8Prep p, const flo
     return;
   }
   if (which == 1) {
-    if (threadIdx.x < 128) {
-      float sum = 0.f;
-      if (p.smooth_k)
-        for (int c = 0; c < kChunks; ++c) sum += partial[(static_cast<int64_t>(bh) * kChunks + c) * 128 + threadIdx.x];
-      const float m = sum / static_cast<float>(p.N);
-      mean[threadIdx.x] = m;
-      if (blk == 0) p.k_mean[bh * 128 + threadIdx.x] = m;
-    }
+    if (threadIdx.x < 128) mean[threadIdx.x] = p.k_mean[bh * 128 + threadIdx.x];
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -224,8 +232,11 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
   kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  kmean_finalize<<<p.B * p.H, 128, 0, stream>>>(p, partial);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   dim3 g2((p.N + 127) / 128, p.B * p.H, 3);
-  quantize_qkv<<<g2, kThreads, 0, stream>>>(p, partial);
+  quantize_qkv<<<g2, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
