@@ -18,6 +18,12 @@
 //   warps 10-11 idle (they complete the third warpgroup for the register re-split)
 // Registers: launched at 168 per thread; the third warpgroup drops to kRegsAux and
 // the softmax warpgroups rise to kRegsSoftmax (2*128*kRegsSoftmax + 128*kRegsAux <= 64K).
+// BF16: RoPE of Q happens as Q is loaded: the softmax warpgroup that owns a Q
+// tile rotates the raw bf16 rows in shared memory with the cos/sin tables and
+// writes them back in place before the first MMA reads them.  K is rotated once
+// per head by a separate pass, since every CTA of the head re-reads each K tile.
+// FP8: Q, K and V arrive rotated, smoothed (K) and quantised from one prologue
+// pass (rotating and quantising Q here measured 4 % slower per tile).
 // TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256) O0, O1 (d
 // columns each from 256).  P_i (bf16: 64 columns, e4m3: 32) overwrites the
 // first columns of S_i once the softmax has read S_i.
@@ -57,7 +63,7 @@ struct AttnCfg {
   static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
   static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
   static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2;
   static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 16;
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
@@ -74,6 +80,7 @@ struct AttnCfg {
   static constexpr float kTwoTau = static_cast<float>(1ull << kTau);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kRowBytes % 128 == 0, "token rows must be whole 128-byte swizzle atoms");
+  static_assert(BM == BN, "Q and K/V tiles share the column-block size kSubBytes");
 };
 
 // Scales of the FP8 variant (unused by BF16).
@@ -104,6 +111,64 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
                : "memory");
 }
 
+// BF16 Q tile rotation by the softmax warpgroup that owns the tile (128
+// threads): each row is rotated in fp32 with the cos/sin tables and written
+// back in place as bf16 (the tensor-core operand, rounded once).
+// Work split: thread t owns 16-byte channel chunk c = t % CPR (8 channels, 4
+// rotary pairs) of rows t / CPR + RPP k, so a warp reads whole table rows (512
+// contiguous bytes per load instruction).  Every table load is issued before the
+// wait for the tile (the caller passes the wait in as a callable), so one L2
+// round trip overlaps the TMA load; a thread-per-row split with per-chunk loads
+// serialised sixteen round trips (about 16k cycles per CTA, measured).
+// Out of line, so that its registers stay out of the softmax branch's allocation.
+template <int D, typename Wait>
+__device__ __noinline__ void rotate_q_tile(uint8_t* q_tile, const float* rope_cos, const float* rope_sin, int qrow0,
+                                           int N, Wait wait_tile) {
+  constexpr int kSubBytes = 128 * 128;  // one 128-row, 128-byte column block
+  constexpr int CPR = D / 8;            // 16-byte chunks per row
+  constexpr int RPP = 128 / CPR;        // rows covered per pass
+  constexpr int NP = 128 / RPP;         // passes (= rows per thread)
+  const int t = threadIdx.x & 127;
+  const int c = t % CPR, r0 = t / CPR;
+  const bool rope = rope_cos != nullptr;
+  float4 cv[NP], sv[NP];
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    const int n = qrow0 + r0 + RPP * k;
+    if (rope && n < N) {  // rows past N are zero-filled by TMA and stay 0
+      cv[k] = __ldg(reinterpret_cast<const float4*>(rope_cos + static_cast<int64_t>(n) * (D / 2)) + c);
+      sv[k] = __ldg(reinterpret_cast<const float4*>(rope_sin + static_cast<int64_t>(n) * (D / 2)) + c);
+    } else {
+      cv[k] = make_float4(1.f, 1.f, 1.f, 1.f);
+      sv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  const bool q_ok = wait_tile();
+  if (!rope || !q_ok) return;
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    // row r's chunk c sits at column block c / 8, 16-byte slot (c % 8) ^ (r % 8) (128-byte swizzle)
+    const int r = r0 + RPP * k;
+    uint4* p = reinterpret_cast<uint4*>(q_tile + r * 128 + (c >> 3) * kSubBytes + (((c & 7) ^ (r & 7)) << 4));
+    const uint4 xv = *p;
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
+    const float cc[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w}, ss[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(xp[e]);
+      y[2 * e] = x.x * cc[e] - x.y * ss[e];
+      y[2 * e + 1] = x.x * ss[e] + x.y * cc[e];
+    }
+    uint4 o4;
+    o4.x = pack_bf16x2(y[0], y[1]);
+    o4.y = pack_bf16x2(y[2], y[3]);
+    o4.z = pack_bf16x2(y[4], y[5]);
+    o4.w = pack_bf16x2(y[6], y[7]);
+    *p = o4;
+  }
+}
+
 template <bool FP8, int D>
 __global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -122,6 +187,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_empty = v_full + NV;
   uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and every earlier MMA)
   uint64_t* pv_done = s_full + 2;    // [2] PV_i(j) computed (read by the epilogue)
+  uint64_t* q_ready = pv_done + 2;   // [2] BF16: Q_i rotated in shared memory (128 arrivals)
   // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
   //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
   constexpr uint32_t kBarPReady = 1, kBarTurn = 3;
@@ -139,6 +205,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(q_full + i, 1);
       mbar_init(s_full + i, 1);
       mbar_init(pv_done + i, 1);
+      mbar_init(q_ready + i, 128);
     }
     for (int s = 0; s < NK; ++s) {
       mbar_init(k_full + s, 1);
@@ -224,7 +291,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
       const bool leader = lane == 0;
-      bool ok = mbar_wait(q_full, 0, err, kErrTimeout) && mbar_wait(k_full, 0, err, kErrTimeout);
+      uint64_t* q_in = FP8 ? q_full : q_ready;  // BF16 waits for the in-place rotation
+      bool ok = mbar_wait(q_in, 0, err, kErrTimeout) && mbar_wait(k_full, 0, err, kErrTimeout);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
@@ -233,7 +301,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(s_full);
           mma_commit(k_empty);
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(q_full + 1, 0, err, kErrTimeout));
+        ok = __all_sync(0xffffffffu, mbar_wait(q_in + 1, 0, err, kErrTimeout));
       }
       if (ok) {
         tc_fence_after();
@@ -282,12 +350,24 @@ __global__ void __launch_bounds__(384, 1)
     regs_inc<C::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     const int i = warp >> 2;                    // Q tile of this warpgroup
+    const int qblk = 2 * qt + i;                // 128-row block index of this Q tile
+    // ------------------------------------------------ BF16: rotate Q on load
+    // First, while almost nothing is live: the per-tile loop's constants are formed
+    // after it, so the preparation's registers cannot push them into local memory
+    // (measured: 6 % slower per tile when it ran after them).
+    if constexpr (!FP8) {
+      uint64_t* qf = q_full + i;
+      auto wait_tile = [qf, err]() { return mbar_wait(qf, 0, err, kErrTimeout); };
+      rotate_q_tile<D>(sQ + i * C::kTileBytes, out.rope_cos, out.rope_sin, qblk * BM, N, wait_tile);
+      // the MMA reads Q through the async proxy: order the generic-proxy writes first
+      fence_proxy_async_smem();
+      mbar_arrive(q_ready + i);
+    }
     const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + C::kColS + 128 * i + lane_off;
     const uint32_t tO = tmem + C::kColO + D * i + lane_off;
     const float sl2 = out.scale_log2;
-    const int qblk = 2 * qt + i;                // 128-row block index of this Q tile
     // FP8 scales: score = S * sQ * sK(j) * scale, P8 = p * 2^-tau * 448 * sV(j) / sV_max
     float qs = sl2, vfold = 1.f, fin_scale = 1.f;
     const float* ksc = nullptr;

@@ -158,7 +158,7 @@ dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d, const 
 
 size_t dit_attn_bf16_workspace_bytes(int B, int H, int N, int d, int has_rope) {
   if (!has_rope || B < 1 || H < 1 || N < 1 || d < 1) return 0;
-  return 2 * align256(static_cast<size_t>(B) * H * N * d * 2);
+  return align256(static_cast<size_t>(B) * H * N * d * 2);  // rotated K
 }
 
 dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
@@ -180,31 +180,28 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
   if (!ds || !ds->sm100 || !g_encode) return DIT_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  const void* qa = q;
   const void* ka = k;
-  int64_t sqa[3] = {sq[0], sq[1], sq[2]}, ska[3] = {sk[0], sk[1], sk[2]};
+  int64_t ska[3] = {sk[0], sk[1], sk[2]};
   if (rope) {
-    // Rotated Q and K are staged contiguously in the workspace.
-    uint8_t* w = static_cast<uint8_t*>(workspace);
-    void* qr = w;
-    void* kr = w + need / 2;
+    // K is rotated once per head into the workspace (every CTA of the head reads
+    // each K tile); Q is rotated by the attention kernel as it loads each Q tile.
+    void* kr = workspace;
     const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
-    dit::RopeJob jobs[2];
-    jobs[0].x = q; jobs[0].y = qr;
-    jobs[1].x = k; jobs[1].y = kr;
+    dit::RopeJob job;
+    job.x = k;
+    job.y = kr;
     for (int i = 0; i < 3; ++i) {
-      jobs[0].sx[i] = sq[i]; jobs[0].sy[i] = cs[i];
-      jobs[1].sx[i] = sk[i]; jobs[1].sy[i] = cs[i];
+      job.sx[i] = sk[i];
+      job.sy[i] = cs[i];
     }
-    cudaError_t e = dit::launch_rope_apply(jobs, 2, B, H, N, d, rope_cos, rope_sin, 0, st);
+    cudaError_t e = dit::launch_rope_apply(&job, 1, B, H, N, d, rope_cos, rope_sin, 0, st);
     if (e != cudaSuccess) return DIT_ERR_LAUNCH;
-    qa = qr;
     ka = kr;
-    for (int i = 0; i < 3; ++i) sqa[i] = ska[i] = cs[i];
+    for (int i = 0; i < 3; ++i) ska[i] = cs[i];
   }
   CUtensorMap tq, tk, tv;
   // Q tiles are 128 tokens, K/V tiles kAttnBlockN tokens; boxes are 128 bytes wide.
-  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qa, B, H, N, d, sqa, 64, 128) ||
+  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, B, H, N, d, sq, 64, 128) ||
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ka, B, H, N, d, ska, 64, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, B, H, N, d, sv, 64, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
@@ -215,6 +212,8 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   out.scale_log2 = scale * 1.4426950408889634f;
   out.err = ds->err;
+  out.rope_cos = rope_cos;
+  out.rope_sin = rope_sin;
   return launch_status(dit::launch_attn_bf16(tq, tk, tv, out, B, H, d, st));
 }
 
@@ -281,6 +280,8 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   out.scale_log2 = scale * 1.4426950408889634f;
   out.err = ds->err;
+  out.rope_cos = nullptr;  // Q arrives rotated and quantised from the prologue
+  out.rope_sin = nullptr;
   return launch_status(dit::launch_attn_fp8(tq, tk, tv, out, p, st));
 }
 

@@ -42,6 +42,11 @@ struct AttnOut {
   int N;
   float scale_log2;  // softmax scale * log2(e)
   int* err;          // device error word
+  // BF16 only: fp32 [N][d/2] rotary tables for Q, applied as the attention
+  // kernel loads Q (both null: Q is used as given).  FP8 takes Q rotated and
+  // quantised by its prologue.
+  const float* rope_cos;
+  const float* rope_sin;
 };
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,

@@ -106,7 +106,9 @@ DIT_API dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d
 /* ------------------------------------------------------------------------ */
 
 /* Workspace needed by dit_attn_bf16 (0 when has_rope == 0).  With rotary
- * tables the rotated Q and K are staged there as contiguous bf16 [B,H,N,d]. */
+ * tables the rotated K is staged there as contiguous bf16 [B,H,N,d] (one pass
+ * per call; every Q tile reads every K tile).  Q is rotated inside the
+ * attention kernel as each Q tile is loaded and needs no workspace. */
 DIT_API size_t dit_attn_bf16_workspace_bytes(int B, int H, int N, int d, int has_rope);
 
 /* O = attention(Q, K, V) in BF16 with fp32 accumulation and softmax.
@@ -121,10 +123,12 @@ DIT_API dit_status dit_attn_bf16(const void* q, const void* k, const void* v, vo
                          size_t workspace_bytes, dit_stream_t stream);
 
 /* Workspace needed by dit_attn_fp8: e4m3 copies of rotated Q, smoothed K
- * and V, their per-block fp32 scales and the fp32 K channel means. */
+ * and V, their per-block fp32 scales and the fp32 K channel means (one
+ * prologue pass rotates, smooths and quantises them before the attention
+ * kernel runs). */
 DIT_API size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_block, int kv_block);
 
-/* O = attention in FP8: Q, K, V rotated (Q, K), K smoothed (smooth_k != 0:
+/* O = attention in FP8: Q and K rotated, K smoothed (smooth_k != 0:
  * per-(b,h) channel mean over all N tokens subtracted after rotation), then
  * quantised to e4m3 (RNE, saturating) with one fp32 scale amax/448 per block
  * of q_block (Q) or kv_block (K, V) tokens.  Scores accumulate in fp32; P is

@@ -55,7 +55,7 @@ def test_attention_argument_validation():
     assert _attn(L, cos=A16) == 3                     # only one of the two tables
     assert _attn(L, cos=A16, sin=A16) == 4            # RoPE needs a workspace
     need = L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 1)
-    assert need == 2 * (2 * 16 * 64)                 # rotated Q and K, bf16, 256-byte aligned
+    assert need == 2 * 16 * 64                       # rotated K, bf16, 256-byte aligned (Q rotates in-kernel)
     assert _attn(L, cos=A16, sin=A16, ws=A16, wsb=need - 1) == 4
     assert L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 0) == 0
 
