@@ -76,6 +76,10 @@ struct AttnCfg {
   // at the price of smaller P codes; at tau = 4 only p < 2^-11 (relative to the
   // row max) falls below the e4m3 normal range.
   static constexpr int kTau = FP8 ? 4 : 8;
+  // BF16 hands P to the MMA warp in two 64-key halves, so that the first half of
+  // PV runs while the second half is exponentiated (2.3 % fewer cycles); for FP8,
+  // whose PV is only four MMAs, the extra hand-off costs more than it hides (+7 %).
+  static constexpr bool kSplitP = !FP8;
   static constexpr float kRescaleLog2 = static_cast<float>(kTau);
   static constexpr float kTwoTau = static_cast<float>(1ull << kTau);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -190,7 +194,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* q_ready = pv_done + 2;   // [2] BF16: Q_i rotated in shared memory (128 arrivals)
   // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
   //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
-  constexpr uint32_t kBarPReady = 1, kBarTurn = 3;
+  //                 kBarPHalf + i   BF16: softmax i stored keys 0..63 of P (128 arrive, MMA warp syncs)
+  constexpr uint32_t kBarPReady = 1, kBarTurn = 3, kBarPHalf = 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
 
   const int warp = threadIdx.x >> 5;
@@ -277,17 +282,19 @@ __global__ void __launch_bounds__(384, 1)
             mma_f16_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      auto pv = [&](int i, int sv, bool acc) {  // O_i (+)= P_i V
+      // O_i (+)= P_i V over MMA steps [k0, k1) of the tile's keys; the first step
+      // overwrites O_i when acc is false (first tile)
+      auto pv = [&](int i, int sv, bool acc, int k0, int k1) {
         const uint32_t va = v_addr + sv * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < BN / C::kKStep; ++kk) {
+        for (int kk = k0; kk < k1; ++kk) {
           // kKStep keys = kKStep rows of 128 bytes; d column blocks are kSubBytes apart
           const uint64_t bd = smem_desc_sw128(va + kk * C::kKStep * 128, C::kSubBytes, 1024);
           const uint32_t pa = tmem + C::kColS + 128 * i + kk * 8;  // 8 columns of packed P per MMA
           if constexpr (FP8)
-            mma_f8_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+            mma_f8_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
           else
-            mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+            mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
         }
       };
       const bool leader = lane == 0;
@@ -318,10 +325,17 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout);
         if (ok && j < nkv) ok = mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout);
         if (!__all_sync(0xffffffffu, ok)) break;
+        constexpr int NKK = BN / C::kKStep, KH = C::kSplitP ? NKK / 2 : 0;
+        if constexpr (C::kSplitP) {  // first half of PV_0 while softmax 0 finishes P_0
+          named_sync<kBarPHalf + 0, 160>();
+          tc_fence_after();
+          if (leader) pv(0, sv, jj > 0, 0, KH);
+          __syncwarp();
+        }
         named_sync<kBarPReady + 0, 160>();
         tc_fence_after();
         if (leader) {
-          pv(0, sv, jj > 0);
+          pv(0, sv, KH > 0 || jj > 0, KH, NKK);
           mma_commit(pv_done);
           mma_commit(v_empty + sv);
           if (j < nkv) {
@@ -331,10 +345,16 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         __syncwarp();
+        if constexpr (C::kSplitP) {
+          named_sync<kBarPHalf + 1, 160>();
+          tc_fence_after();
+          if (leader) pv(1, sv, jj > 0, 0, KH);
+          __syncwarp();
+        }
         named_sync<kBarPReady + 1, 160>();
         tc_fence_after();
         if (leader) {
-          pv(1, sv, jj > 0);
+          pv(1, sv, KH > 0 || jj > 0, KH, NKK);
           mma_commit(pv_done + 1);
           mma_commit(v_empty + sv);
           if (j < nkv) {
@@ -384,6 +404,32 @@ __global__ void __launch_bounds__(384, 1)
       vfold = 448.f / (vmax * C::kTwoTau);
       fin_scale = vmax * C::kTwoTau / 448.f;
     }
+    // O_i *= alpha, RC columns at a time (64 while half of the scores are still in
+    // registers, all d after the tile's exps).  Called once S_i(j) is seen complete:
+    // the commit behind it covers PV_i(0..j-1), so no MMA is writing O_i.
+    auto rescale_o = [&](float alpha) {
+      constexpr int RC = C::kSplitP ? 64 : D;
+      const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll
+      for (int hc = 0; hc < D / RC; ++hc) {
+        uint32_t o[RC];
+#pragma unroll
+        for (int c = 0; c < RC / 32; ++c) tmem_ld32(tO + hc * RC + c * 32, o + c * 32);
+        tmem_wait_ld();
+        reg_fence(o);
+#pragma unroll
+        for (int e = 0; e < RC / 2; ++e) {
+          float x, y;
+          f2_split(fmul2(f2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), a2), x, y);
+          o[2 * e] = __float_as_uint(x);
+          o[2 * e + 1] = __float_as_uint(y);
+        }
+#pragma unroll
+        for (int c = 0; c < RC / 32; ++c) tmem_st32(tO + hc * RC + c * 32, o + c * 32);
+        tmem_wait_st();
+        reg_fence(o);
+      }
+    };
     float m = -INFINITY;  // running (possibly stale) max of the scaled log2 scores
     float l = 0.f;
     bool ok = true;
@@ -475,6 +521,14 @@ __global__ void __launch_bounds__(384, 1)
             p[16 * q + e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + 16 * q, p + 16 * q);
+          if (C::kSplitP && q == 1) {  // keys 0..63 of P are in TMEM: PV may start on them once O is rescaled
+            tmem_wait_st();
+            reg_fence(p);
+            if (j > 0 && grow) rescale_o(alpha);
+            tc_fence_before();
+            if (i == 0) named_arrive<kBarPHalf + 0, 160>();
+            else named_arrive<kBarPHalf + 1, 160>();
+          }
         }
       }
       // every arrive is matched by a sync of the other warpgroup
@@ -482,25 +536,7 @@ __global__ void __launch_bounds__(384, 1)
       else if (j + 1 < nkv) named_arrive<kBarTurn + 0, 256>();
       tmem_wait_st();
       reg_fence(p);
-      if (j > 0 && grow) {  // O_i holds PV_i(0..j-1): the commit behind S_i(j) covers them
-        uint32_t o[D];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o + c * 32);
-        tmem_wait_ld();
-        reg_fence(o);
-        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll
-        for (int e = 0; e < D / 2; ++e) {
-          float x, y;
-          f2_split(fmul2(f2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), a2), x, y);
-          o[2 * e] = __float_as_uint(x);
-          o[2 * e + 1] = __float_as_uint(y);
-        }
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_st32(tO + c * 32, o + c * 32);
-        tmem_wait_st();
-        reg_fence(o);
-      }
+      if (!C::kSplitP && j > 0 && grow) rescale_o(alpha);
       tc_fence_before();
       if (i == 0) named_arrive<kBarPReady + 0, 160>();
       else named_arrive<kBarPReady + 1, 160>();
