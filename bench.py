@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel, keyed
 # by the hash of the kernel source it was taken on; a changed kernel reports null.
 NCU_TRAFFIC = {
-    # profiles/attn_bf16_flux2k.md: 323.0 MB read + 87.4 MB written per launch
-    ("attn_bf16", "4b071d3b8e2cd485"): 410_338_304,
+    # profiles/attn_bf16_flux2k.md: 326.7 MB read + 89.2 MB written per launch
+    ("attn_bf16", "e3a5346cb92e8aa8"): 415_904_256,
 }
 
 
