@@ -36,7 +36,9 @@
 // V stages are freed by count-2 mbarriers with one commit after each of the two
 // MMAs reading the stage.  The tensor core runs PV1(j-1), S1(j) while softmax 0
 // works on S0(j), and PV0(j), S0(j+1) while softmax 1 works on S1(j); the two
-// softmax warpgroups take turns on the ex2 unit.  Thread-to-thread hand-offs
+// softmax warpgroups take turns on the ex2 unit.  BF16 releases P_i(j) in two
+// 64-key halves, so the MMA thread issues the first half of PV_i(j) while the
+// second half is still being exponentiated.  Thread-to-thread hand-offs
 // (P ready -> MMA warp, the ping-pong turns) use named barriers, which are
 // far cheaper than an mbarrier round trip; mbarriers remain only where the
 // tensor core or the TMA unit signals.
