@@ -525,6 +525,47 @@ def run_trace(args):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8_peak():
+    """Dense e4m3 GEMM throughput of the library (cuBLASLt through torch._scaled_mm),
+    8192^3, bf16 output: best of 10 (burst) and back to back for 4 s (sustained).
+    A denominator for the FP8 attention, measured the way the bf16 peak is."""
+    import torch
+    n = 8192
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(7)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()  # column-major operand
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    flops = 2.0 * n ** 3
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    with ClockSampler(0) as clk:
+        reps, t_end = 0, time.time() + 4.0
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        while time.time() < t_end:
+            for _ in range(20):
+                mm()
+            reps += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+    sustained = flops * reps / (e0.elapsed_time(e1) / 1e3) / 1e12
+    print(json.dumps({"fp8_e4m3_tflops": flops / (best / 1e3) / 1e12, "fp8_e4m3_tflops_sustained": sustained,
+                      "how": "torch._scaled_mm e4m3 8192^3, bf16 out, unit scales: best of 10 / 4 s loop",
+                      "clocks": clk.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,6 +575,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--trace", action="store_true", help="run the 28-step denoising trace instead")
+    ap.add_argument("--measure-fp8-peak", action="store_true", help="dense e4m3 GEMM peak (a denominator) instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -545,6 +587,9 @@ def main():
         return
     if args.trace:
         run_trace(args)
+        return
+    if args.measure_fp8_peak:
+        run_fp8_peak()
         return
     if world > 1:
         import datetime
