@@ -37,6 +37,10 @@ WORKLOAD = "flux2k"
 HIDDEN = 3072
 THRESHOLD = 0.12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Dense e4m3 GEMM (cuBLASLt via torch._scaled_mm, 8192^3) measured on this machine with
+# `python bench.py --measure-fp8-peak` (profiles/fp8_gemm_peak.md); reported beside
+# the nominal-ratio FP8 peak, which stays the roofline denominator.
+FP8_GEMM_MEASURED = {"burst": 3132.4, "sustained": 2594.0}
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel, keyed
 # by the hash of the kernel source it was taken on (code only, comments ignored);
@@ -331,7 +335,10 @@ def run_ours(args, rank, world, local_rank):
         fp8 = {"value": v8 / 1e12, "unit": "TFLOP/s", "ms_per_step": mps8,
                "peak": fp8_peak, "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
                "frac_of_step": v8 / 1e12 / fp8_peak,
-               "peak_sustained": fp8_sus, "frac_of_step_vs_sustained": v8 / 1e12 / fp8_sus}
+               "peak_sustained": fp8_sus, "frac_of_step_vs_sustained": v8 / 1e12 / fp8_sus,
+               "measured_fp8_gemm": FP8_GEMM_MEASURED,
+               "frac_of_step_vs_measured_fp8_gemm": v8 / 1e12 / FP8_GEMM_MEASURED["burst"],
+               "frac_of_step_vs_measured_fp8_gemm_sustained": v8 / 1e12 / FP8_GEMM_MEASURED["sustained"]}
         assert dit.read_error() == 0
 
     # ---- e2e through the public API from pinned host buffers.  Every step copies its
