@@ -15,4 +15,5 @@ from ._binding import (  # noqa: F401
     read_error,
     rope_apply,
     rope_tables,
+    selftest_wait_timeout,
 )

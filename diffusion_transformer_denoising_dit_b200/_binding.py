@@ -19,7 +19,8 @@ STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "D
           4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT"}
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
-           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc"]
+           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
+           "dit_selftest_wait_timeout"]
 
 
 class DitError(RuntimeError):
@@ -48,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.dit_status_string.argtypes = [_i]
         L.dit_read_error.restype = _i
         L.dit_read_error.argtypes = [_vp]
+        L.dit_selftest_wait_timeout.restype = _i
+        L.dit_selftest_wait_timeout.argtypes = [_vp]
         L.dit_rope_tables.restype = _i
         L.dit_rope_tables.argtypes = [_vp, _i, _i, _i, _i, ctypes.c_double, _vp, _vp, _vp]
         L.rope_apply.restype = _i
@@ -104,6 +107,14 @@ def read_error(stream=None) -> int:
     """Synchronise the stream and return+clear the device error word (0 = none)."""
     s = torch.cuda.current_stream().cuda_stream if stream is None else stream
     return lib().dit_read_error(s)
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the failure-detection self test: a bounded wait that nothing
+    satisfies, which gives up after its limit and records DIT_ERR_TIMEOUT
+    (read it with read_error())."""
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    _check("dit_selftest_wait_timeout", lib().dit_selftest_wait_timeout(s))
 
 
 def rope_tables(pos: torch.Tensor, axes, theta: float = 10000.0):

@@ -122,6 +122,12 @@ dit_status dit_read_error(dit_stream_t stream) {
   return static_cast<dit_status>(v);
 }
 
+dit_status dit_selftest_wait_timeout(dit_stream_t stream) {
+  const DeviceState* ds = device_state();
+  if (!ds || !ds->sm100 || !ds->err) return DIT_ERR_UNSUPPORTED;
+  return launch_status(dit::launch_selftest_wait(ds->err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, double theta, float* cos_out,
                            float* sin_out, dit_stream_t stream) {
   if (!pos || !cos_out || !sin_out || N < 1) return DIT_ERR_INVALID_ARG;

@@ -79,6 +79,9 @@ constexpr int kFp8MeanChunks = 48;
 
 cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream);
 
+// One thread waits (bounded) on an mbarrier nothing arrives on: records kErrTimeout.
+cudaError_t launch_selftest_wait(int* err, cudaStream_t stream);
+
 cudaError_t launch_attn_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
                             const Fp8Prep& p, cudaStream_t stream);
 

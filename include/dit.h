@@ -84,6 +84,14 @@ DIT_API const char* dit_status_string(dit_status s);
  * current device (DIT_OK if no kernel recorded a failure). */
 DIT_API dit_status dit_read_error(dit_stream_t stream);
 
+/* Failure-detection self test (no counterpart on the pages; it exercises the
+ * library's own error path).  Enqueues one thread that waits, through the
+ * bounded wait every kernel uses, on a barrier that nothing arrives on: after
+ * the wait limit (1 s) it records DIT_ERR_TIMEOUT in the device error word and
+ * ends, leaving the context usable.  dit_read_error then returns
+ * DIT_ERR_TIMEOUT.  Returns DIT_ERR_UNSUPPORTED off sm_100. */
+DIT_API dit_status dit_selftest_wait_timeout(dit_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Rotary embedding                                                          */
 /* ------------------------------------------------------------------------ */
