@@ -142,7 +142,8 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
     if (two_blocks) *sc_out1 = s1;
     if (vmax) {
       atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s0));
-      if (two_blocks) atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s1));
+      // a second block past the sequence end (all zeros, scale 1) is not a V block
+      if (two_blocks && n_base + 64 < N) atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s1));
     }
   }
 #pragma unroll
