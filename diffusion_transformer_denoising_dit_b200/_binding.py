@@ -20,7 +20,7 @@ STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
            "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
-           "dit_selftest_wait_timeout"]
+           "dit_selftest_wait_timeout", "dit_attn_bf16_skippable"]
 
 
 class DitError(RuntimeError):
@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_bf16.restype = _i
         L.dit_attn_bf16.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _i64x3, _i64x3,
                                     _vp, _vp, ctypes.c_float, _vp, _sz, _vp]
+        L.dit_attn_bf16_skippable.restype = _i
+        L.dit_attn_bf16_skippable.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _i64x3, _i64x3,
+                                              _vp, _vp, ctypes.c_float, _vp, _sz, _vp, _vp]
         L.dit_attn_fp8_workspace_bytes.restype = _sz
         L.dit_attn_fp8_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
         L.dit_attn_fp8.restype = _i
@@ -147,9 +150,16 @@ def rope_apply(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, out_dtype=
 
 
 def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float | None = None,
-              out=None, workspace=None, q_block: int = 128, kv_block: int = 64, smooth_k: bool = True):
-    """Joint attention O [B,H,N,d] bf16 from bf16 q, k, v (+ optional rotary tables)."""
-    _need_cuda(q, k, v, cos, sin)
+              out=None, workspace=None, q_block: int = 128, kv_block: int = 64, smooth_k: bool = True,
+              skip=None):
+    """Joint attention O [B,H,N,d] bf16 from bf16 q, k, v (+ optional rotary tables).
+
+    skip (BF16 only): a device int32 flag, e.g. FBCacheGate's output; when it is
+    non-zero at the time the kernels run, the call does nothing and ``out`` keeps
+    its previous contents."""
+    _need_cuda(q, k, v, cos, sin, skip)
+    if skip is not None and (precision != "bf16" or skip.dtype != torch.int32 or skip.numel() < 1):
+        raise ValueError("skip must be a CUDA int32 flag and is supported for precision='bf16'")
     for t in (q, k, v):
         if t.dtype != torch.bfloat16:
             raise ValueError("q, k, v must be bf16")
@@ -172,7 +182,9 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
     wb = need if need else 0
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
             _strides(q), _strides(k), _strides(v), _strides(out), _ptr(cos), _ptr(sin), sc)
-    if precision == "bf16":
+    if precision == "bf16" and skip is not None:
+        _check("dit_attn_bf16_skippable", L.dit_attn_bf16_skippable(*args, wp, wb, skip.data_ptr(), _stream(q)))
+    elif precision == "bf16":
         _check("dit_attn_bf16", L.dit_attn_bf16(*args, wp, wb, _stream(q)))
     else:
         _check("dit_attn_fp8", L.dit_attn_fp8(*args, q_block, kv_block, int(smooth_k), wp, wb, _stream(q)))

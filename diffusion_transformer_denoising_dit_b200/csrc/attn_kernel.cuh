@@ -186,6 +186,9 @@ __global__ void __launch_bounds__(384, 1)
                 const __grid_constant__ CUtensorMap tmV, const AttnOut out, const AttnScales sc) {
   using C = AttnCfg<FP8, D>;
   constexpr int NK = C::NK, NV = C::NV, BM = C::BM, BN = C::BN;
+  // device-side skip (the cache gate's flag): the whole CTA leaves before any
+  // barrier, TMEM allocation or load, so an early return is safe
+  if (out.skip != nullptr && *out.skip != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // Q0, Q1

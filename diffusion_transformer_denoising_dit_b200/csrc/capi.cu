@@ -167,10 +167,12 @@ size_t dit_attn_bf16_workspace_bytes(int B, int H, int N, int d, int has_rope) {
   return align256(static_cast<size_t>(B) * H * N * d * 2);  // rotated K
 }
 
-dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
-                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
-                         const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
-                         size_t workspace_bytes, dit_stream_t stream) {
+namespace {
+
+dit_status attn_bf16_impl(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                          const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                          const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
+                          size_t workspace_bytes, const int32_t* skip, dit_stream_t stream) {
   if (!q || !k || !v || !o || !sq || !sk || !sv || !so) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return DIT_ERR_INVALID_ARG;
@@ -200,7 +202,7 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
       job.sx[i] = sk[i];
       job.sy[i] = cs[i];
     }
-    cudaError_t e = dit::launch_rope_apply(&job, 1, B, H, N, d, rope_cos, rope_sin, 0, st);
+    cudaError_t e = dit::launch_rope_apply(&job, 1, B, H, N, d, rope_cos, rope_sin, 0, st, skip);
     if (e != cudaSuccess) return DIT_ERR_LAUNCH;
     ka = kr;
     for (int i = 0; i < 3; ++i) ska[i] = cs[i];
@@ -211,7 +213,7 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ka, B, H, N, d, ska, 64, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, B, H, N, d, sv, 64, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
-  dit::AttnOut out;
+  dit::AttnOut out{};  // value-initialised: every pointer not set below is null
   out.o = o;
   for (int i = 0; i < 3; ++i) out.so[i] = so[i];
   out.N = N;
@@ -220,7 +222,29 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
   out.err = ds->err;
   out.rope_cos = rope_cos;
   out.rope_sin = rope_sin;
+  out.skip = skip;
   return launch_status(dit::launch_attn_bf16(tq, tk, tv, out, B, H, d, st));
+}
+
+}  // namespace
+
+dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                         const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
+                         size_t workspace_bytes, dit_stream_t stream) {
+  return attn_bf16_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, workspace,
+                        workspace_bytes, nullptr, stream);
+}
+
+dit_status dit_attn_bf16_skippable(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                                   const int64_t sq[3], const int64_t sk[3], const int64_t sv[3],
+                                   const int64_t so[3], const float* rope_cos, const float* rope_sin,
+                                   float softmax_scale, void* workspace, size_t workspace_bytes,
+                                   const int32_t* skip, dit_stream_t stream) {
+  if (!skip) return DIT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(skip) & 3u) return DIT_ERR_ALIGNMENT;
+  return attn_bf16_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, workspace,
+                        workspace_bytes, skip, stream);
 }
 
 size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_block, int kv_block) {
@@ -279,7 +303,7 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.k8, B, H, N, d, cs, 128, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.v8, B, H, N, d, cs, 128, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
-  dit::AttnOut out;
+  dit::AttnOut out{};  // value-initialised: every pointer not set below is null
   out.o = o;
   for (int i = 0; i < 3; ++i) out.so[i] = so[i];
   out.N = N;

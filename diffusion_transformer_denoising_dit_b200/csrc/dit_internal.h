@@ -28,9 +28,11 @@ struct RopeJob {
   int64_t sy[3];
 };
 
-// Applies rotary embedding to njobs (1 or 2) tensors of the same shape in one launch.
+// Applies rotary embedding to njobs (1 or 2) tensors of the same shape in one launch
+// (nothing when skip is non-null and *skip != 0 at execution time).
 cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int N, int d, const float* cos_tab,
-                              const float* sin_tab, int out_fp32, cudaStream_t stream);
+                              const float* sin_tab, int out_fp32, cudaStream_t stream,
+                              const int32_t* skip = nullptr);
 
 cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold, float* rel_out, int32_t* skip_out,
                         double* partials, cudaStream_t stream);
@@ -47,6 +49,8 @@ struct AttnOut {
   // quantised by its prologue.
   const float* rope_cos;
   const float* rope_sin;
+  // when non-null and *skip != 0 at execution time the launch does nothing
+  const int32_t* skip;
 };
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,

@@ -50,6 +50,7 @@ struct RopeArgs {
   const float* cos_tab;
   const float* sin_tab;
   int out_fp32;
+  const int32_t* skip;  // non-null and set: do nothing
 };
 
 // One thread per 8 consecutive channels (4 pairs): one 16-byte load of x, two
@@ -58,6 +59,7 @@ struct RopeArgs {
 // covers every chunk once (measured faster than a grid-stride loop or several
 // chunks per thread, which cost occupancy).
 __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
+  if (a.skip != nullptr && *a.skip != 0) return;
   const RopeJob& jb = a.job[blockIdx.y];
   const int cpr = a.d / 8;  // chunks per row
   const int64_t total = static_cast<int64_t>(a.B) * a.H * a.N * cpr;
@@ -99,12 +101,13 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
 }
 
 cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int N, int d, const float* cos_tab,
-                              const float* sin_tab, int out_fp32, cudaStream_t stream) {
+                              const float* sin_tab, int out_fp32, cudaStream_t stream, const int32_t* skip) {
   RopeArgs a;
   for (int i = 0; i < njobs; ++i) a.job[i] = jobs[i];
   if (njobs == 1) a.job[1] = jobs[0];
   a.B = B; a.H = H; a.N = N; a.d = d;
   a.cos_tab = cos_tab; a.sin_tab = sin_tab; a.out_fp32 = out_fp32;
+  a.skip = skip;
   const int64_t total = static_cast<int64_t>(B) * H * N * (d / 8);
   const int64_t blocks = (total + 255) / 256;
   dim3 grid(static_cast<unsigned>(blocks), njobs);

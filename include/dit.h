@@ -130,6 +130,23 @@ DIT_API dit_status dit_attn_bf16(const void* q, const void* k, const void* v, vo
                          const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
                          size_t workspace_bytes, dit_stream_t stream);
 
+/* dit_attn_bf16 whose work is conditional on a device flag: when *skip != 0 at
+ * the time the kernels run, both launches (the K rotation and the attention)
+ * return at once and o is left as it was.  skip: device int32, 4-byte aligned,
+ * typically the skip_out of fbcache_gate on the same stream, so that a
+ * denoising step's remaining blocks can be enqueued without reading the gate's
+ * decision on the host (the device-side form of First-Block-Cache skipping:
+ * unsloth studio commit, "Add opt-in step caching (First-Block-Cache)"; the
+ * decision is otherwise a graph break, as the FLUX 3 / TensorRT-LLM VisualGen
+ * page's CUDA-graph note implies).  Other arguments and errors as
+ * dit_attn_bf16; DIT_ERR_INVALID_ARG for a null skip, DIT_ERR_ALIGNMENT for a
+ * misaligned one. */
+DIT_API dit_status dit_attn_bf16_skippable(const void* q, const void* k, const void* v, void* o, int B, int H, int N,
+                                           int d, const int64_t sq[3], const int64_t sk[3], const int64_t sv[3],
+                                           const int64_t so[3], const float* rope_cos, const float* rope_sin,
+                                           float softmax_scale, void* workspace, size_t workspace_bytes,
+                                           const int32_t* skip, dit_stream_t stream);
+
 /* Workspace needed by dit_attn_fp8: e4m3 copies of rotated Q, smoothed K
  * and V, their per-block fp32 scales and the fp32 K channel means (one
  * prologue pass rotates, smooths and quantises them before the attention

@@ -60,6 +60,14 @@ def test_attention_argument_validation():
     assert L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 0) == 0
 
 
+def test_skippable_attention_argument_validation():
+    L = B.lib()
+    st = S(1024, 1024, 64)
+    args = (A16, A16, A16, A16, 1, 1, 16, 64, st, st, st, st, None, None, 0.0, None, 0)
+    assert L.dit_attn_bf16_skippable(*args, None, None) == 1      # the flag is required
+    assert L.dit_attn_bf16_skippable(*args, A16 + 2, None) == 3   # 4-byte aligned flag
+
+
 def test_fp8_argument_validation():
     L = B.lib()
     st = S(1024 * 128, 1024 * 128, 128)

@@ -149,3 +149,42 @@ def test_repeated_calls_are_bitwise_identical_at_scale(precision):
     for _ in range(12):
         assert torch.equal(dit.attention(q, k, v, cos, sin, precision=precision), ref)
     assert dit.read_error() == 0
+
+
+def test_skippable_call_follows_the_device_flag():
+    """dit_attn_bf16_skippable: flag 0 gives the plain call's output bit for bit;
+    flag 1 leaves the output untouched (both launches return at once)."""
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w, device=DEV)
+    pos = synth.positions(w.T, w.G)
+    cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    ref = dit.attention(q, k, v, cos, sin)
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.full_like(q, 7.0)
+    dit.attention(q, k, v, cos, sin, out=out, skip=flag)
+    assert torch.equal(out, ref)
+    flag.fill_(1)
+    out2 = torch.full_like(q, 7.0)
+    dit.attention(q, k, v, cos, sin, out=out2, skip=flag)
+    assert bool((out2 == 7.0).all())
+    assert dit.read_error() == 0
+
+
+def test_gate_flag_drives_skippable_attention_without_host_reads():
+    """The cache gate's device flag gates the next call on the same stream."""
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w, device=DEV)
+    ref = dit.attention(q, k, v)
+    gate = dit.FBCacheGate(0.08, 288 * 128, device=DEV)
+    for eps, expect_skip in ((1e-4, True), (0.3, False)):
+        cur, prev = synth.gate_pair(288, 128, eps)
+        out = torch.full_like(q, 7.0)
+        flag = gate(cur.to(DEV), prev.to(DEV))
+        dit.attention(q, k, v, out=out, skip=flag)
+        torch.cuda.synchronize()
+        assert bool(flag.item()) == expect_skip
+        if expect_skip:
+            assert bool((out == 7.0).all())
+        else:
+            assert torch.equal(out, ref)
+    assert dit.read_error() == 0
