@@ -46,8 +46,8 @@ FP8_GEMM_MEASURED = {"burst": 3132.4, "sustained": 2594.0}
 # by the hash of the kernel source it was taken on (code only, comments ignored);
 # a changed kernel reports null.
 NCU_TRAFFIC = {
-    # profiles/attn_bf16_flux2k.md: 322.1 MB read + 87.6 MB written per launch
-    ("attn_bf16", "d3f0c6455bd5349f"): 409_624_320,
+    # profiles/attn_bf16_flux2k.md: 323.0 MB read + 87.0 MB written per launch
+    ("attn_bf16", "b620164e5e13027b"): 409_936_384,
 }
 
 
