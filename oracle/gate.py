@@ -13,6 +13,13 @@ readings:
 * sum|r_prev| = 0: rel = 0 if the residuals are identical (skip), else +inf;
 * the previous residual is that of the immediately preceding step (block 0
   runs on every step, so it always exists); step 0 is always computed.
+
+Policy variants (the pages name the knob, not the policy): "consecutive" (the
+reading above) and "last_computed", where a step is compared with the residual
+of the last step whose remaining blocks actually ran (the step the cached
+output belongs to), so that small changes accumulate across skipped steps; and
+a warm-up of steps that are always computed ([FBCache] and [vflash] both
+describe early denoising steps as the ones that must run).
 """
 from __future__ import annotations
 
@@ -49,13 +56,26 @@ def relative_l1_loops(r_cur, r_prev) -> float:
     return num / den
 
 
-def trace_decisions(residuals, threshold: float):
-    """Per-step (rel, skip) over a denoising trace; step 0 is always computed."""
-    out = [(float("nan"), False)]
-    prev = None
+def trace_decisions(residuals, threshold: float, policy: str = "consecutive", warmup: int = 1):
+    """Per-step (rel, skip) over a denoising trace.
+
+    policy "consecutive": step t is compared with step t-1; "last_computed": with
+    the last step that was not skipped.  The first max(warmup, 1) steps are always
+    computed (their rel is still reported from step 1 on).
+    """
+    if policy not in ("consecutive", "last_computed"):
+        raise ValueError(policy)
+    out = []
+    ref = None  # index of the residual step t is compared with
     for t, r in enumerate(residuals):
-        if t > 0:
-            rel = relative_l1(r, prev)
-            out.append((rel, skip(rel, threshold)))
-        prev = r
+        if t == 0:
+            out.append((float("nan"), False))
+            ref = 0
+            continue
+        base = t - 1 if policy == "consecutive" else ref
+        rel = relative_l1(r, residuals[base])
+        s = skip(rel, threshold) and t >= warmup
+        out.append((rel, s))
+        if not s:
+            ref = t
     return out

@@ -140,3 +140,19 @@ def test_gate_trace_decisions_match_oracle():
     assert got == [s for _, s in ref]
     assert sum(got) == 16
     assert dit.read_error() == 0
+
+
+def test_gate_last_computed_policy_matches_oracle():
+    """The last-computed policy (compare with the residual of the last step that ran):
+    the gate kernel, fed the reference the policy picks, reproduces the oracle's decisions."""
+    res = list(synth.drift_residuals(1024, 512, steps=28))
+    ref_dec = G.trace_decisions(res, 0.12, policy="last_computed")
+    gate = dit.FBCacheGate(0.12, res[0].numel())
+    got, ref = [False], 0
+    for t in range(1, 28):
+        s = bool(gate(res[t].to(DEV), res[ref].to(DEV)).item())
+        got.append(s)
+        if not s:
+            ref = t
+    assert got == [s for _, s in ref_dec]
+    assert dit.read_error() == 0

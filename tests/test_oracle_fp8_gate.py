@@ -129,3 +129,60 @@ def test_trace_decisions_follow_drift():
         assert abs(dec[k][0] - sched[k - 1]) < 2e-3 * max(1.0, sched[k - 1] * 10)
     skipped = [k for k, (_, s) in enumerate(dec) if s]
     assert skipped == list(range(12, 28))
+
+
+def _geometric_residuals(c, steps, shape=(16, 8), seed=0):
+    """r_t = (1 + c)^t r_0 in fp64: against a reference k steps back, rel = (1 + c)^k - 1 exactly."""
+    r0 = np.random.default_rng(seed).standard_normal(shape) + 3.0
+    return [r0 * (1.0 + c) ** t for t in range(steps)]
+
+
+def test_policy_consecutive_on_geometric_growth():
+    """Each step changes by c = 0.05 < 0.12: every step after the warm-up is skipped."""
+    res = _geometric_residuals(0.05, 12)
+    dec = gate.trace_decisions(res, 0.12, policy="consecutive")
+    assert [s for _, s in dec] == [False] + [True] * 11
+    for _, (rel, _) in enumerate(dec[1:]):
+        assert abs(rel - 0.05) < 1e-12
+
+
+def test_policy_last_computed_accumulates_until_threshold():
+    """Against the last computed step the change grows as (1.05)^k - 1: 0.05, 0.1025 (skip),
+    0.157625 (compute), so exactly every third step runs."""
+    res = _geometric_residuals(0.05, 13)
+    dec = gate.trace_decisions(res, 0.12, policy="last_computed")
+    computed = [t for t, (_, s) in enumerate(dec) if not s]
+    assert computed == [0, 3, 6, 9, 12]
+    assert abs(dec[3][0] - (1.05 ** 3 - 1.0)) < 1e-12
+    assert abs(dec[4][0] - 0.05) < 1e-12  # the reference moved to step 3
+
+
+def test_policy_warmup_forces_early_steps():
+    res = _geometric_residuals(0.01, 8)
+    dec = gate.trace_decisions(res, 0.12, warmup=5)
+    assert [s for _, s in dec] == [False] * 5 + [True] * 3
+    assert all(abs(rel - 0.01) < 1e-12 for rel, _ in dec[1:])
+
+
+def test_policy_last_computed_on_the_drift_trace():
+    """The decaying drift under the last-computed policy: changes accumulate across
+    skipped steps, so fewer steps are skipped than with consecutive comparison, and
+    every skipped step's accumulated change is below the threshold."""
+    res = list(synth.drift_residuals(96, 64, steps=28))
+    cons = gate.trace_decisions(res, 0.12)
+    last = gate.trace_decisions(res, 0.12, policy="last_computed")
+    n_cons = sum(s for _, s in cons)
+    n_last = sum(s for _, s in last)
+    assert 0 < n_last < n_cons
+    ref = 0
+    for t in range(1, 28):
+        rel, s = last[t]
+        assert abs(rel - gate.relative_l1(res[t], res[ref])) < 1e-15
+        assert s == (rel < 0.12)
+        if not s:
+            ref = t
+
+
+def test_policy_rejects_unknown_name():
+    with pytest.raises(ValueError):
+        gate.trace_decisions([np.ones(3)], 0.1, policy="nope")
