@@ -10,6 +10,8 @@ from ._binding import (  # noqa: F401
     attention,
     attention_workspace,
     fbcache_gate,
+    fbcache_gate_finalize,
+    fbcache_gate_sums,
     fp8_workspace_views,
     lib,
     read_error,

@@ -20,7 +20,7 @@ STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
            "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
-           "dit_selftest_wait_timeout", "dit_attn_bf16_skippable"]
+           "dit_selftest_wait_timeout", "dit_attn_bf16_skippable", "fbcache_gate_sums", "fbcache_gate_finalize"]
 
 
 class DitError(RuntimeError):
@@ -72,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.fbcache_gate_workspace_bytes.argtypes = [ctypes.c_int64]
         L.fbcache_gate.restype = _i
         L.fbcache_gate.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+        L.fbcache_gate_sums.restype = _i
+        L.fbcache_gate_sums.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, _sz, _vp]
+        L.fbcache_gate_finalize.restype = _i
+        L.fbcache_gate_finalize.argtypes = [_vp, ctypes.c_float, _vp, _vp, _vp]
         L.fbcache_gate_noalloc.restype = _i
         L.fbcache_gate_noalloc.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp]
         _lib = L
@@ -246,6 +250,39 @@ def fbcache_gate(r_cur, r_prev, threshold: float, rel_out=None, skip_out=None, w
     _check("fbcache_gate", L.fbcache_gate(r_cur.data_ptr(), r_prev.data_ptr(), n, float(threshold),
                                           rel_out.data_ptr(), skip_out.data_ptr(), workspace.data_ptr(),
                                           workspace.numel() * workspace.element_size(), _stream(r_cur)))
+    return rel_out, skip_out
+
+
+def fbcache_gate_sums(r_cur, r_prev, sums_out=None, workspace=None):
+    """Shard totals (sum |r_cur - r_prev|, sum |r_prev|) as a device float64 [2] tensor."""
+    _need_cuda(r_cur, r_prev)
+    if r_cur.dtype != torch.bfloat16 or r_prev.dtype != torch.bfloat16 or r_cur.shape != r_prev.shape:
+        raise ValueError("r_cur, r_prev must be bf16 tensors of one shape")
+    r_cur, r_prev = r_cur.contiguous(), r_prev.contiguous()
+    n = r_cur.numel()
+    L = lib()
+    need = L.fbcache_gate_workspace_bytes(n)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, device=r_cur.device, dtype=torch.uint8)
+    if sums_out is None:
+        sums_out = torch.empty(2, device=r_cur.device, dtype=torch.float64)
+    _check("fbcache_gate_sums", L.fbcache_gate_sums(r_cur.data_ptr(), r_prev.data_ptr(), n, sums_out.data_ptr(),
+                                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                                    _stream(r_cur)))
+    return sums_out
+
+
+def fbcache_gate_finalize(sums, threshold: float, rel_out=None, skip_out=None):
+    """(rel, skip) device tensors from totals summed across shards."""
+    _need_cuda(sums)
+    if sums.dtype != torch.float64 or sums.numel() < 2:
+        raise ValueError("sums must be a device float64 [2] tensor")
+    if rel_out is None:
+        rel_out = torch.empty(1, device=sums.device, dtype=torch.float32)
+    if skip_out is None:
+        skip_out = torch.empty(1, device=sums.device, dtype=torch.int32)
+    _check("fbcache_gate_finalize", lib().fbcache_gate_finalize(sums.data_ptr(), float(threshold), rel_out.data_ptr(),
+                                                              skip_out.data_ptr(), _stream(sums)))
     return rel_out, skip_out
 
 

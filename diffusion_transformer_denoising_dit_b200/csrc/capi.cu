@@ -333,4 +333,27 @@ dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float 
                                         static_cast<double*>(workspace), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int64_t n, double* sums_out, void* workspace,
+                             size_t workspace_bytes, dit_stream_t stream) {
+  if (!r_cur || !r_prev || !sums_out || n < 1) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(r_cur) || !aligned16(r_prev) || (reinterpret_cast<uintptr_t>(sums_out) & 7u)) return DIT_ERR_ALIGNMENT;
+  const size_t need = fbcache_gate_workspace_bytes(n);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 7u)) return DIT_ERR_WORKSPACE;
+  const DeviceState* ds = device_state();
+  if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
+  return launch_status(dit::launch_gate_sums(r_cur, r_prev, n, sums_out, static_cast<double*>(workspace),
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
+                                 dit_stream_t stream) {
+  if (!sums || !rel_out || !skip_out) return DIT_ERR_INVALID_ARG;
+  if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(sums) & 7u) return DIT_ERR_ALIGNMENT;
+  const DeviceState* ds = device_state();
+  if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
+  return launch_status(dit::launch_gate_finalize(sums, threshold, rel_out, skip_out,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -36,6 +36,12 @@ cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int 
 
 cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold, float* rel_out, int32_t* skip_out,
                         double* partials, cudaStream_t stream);
+// Sharded gate: the totals (sum |a - b|, sum |b|) of one shard, and the decision
+// from totals summed across shards.
+cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* sums_out, double* partials,
+                             cudaStream_t stream);
+cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
+                                 cudaStream_t stream);
 
 // Output description shared by the attention kernels.
 struct AttnOut {

@@ -96,9 +96,10 @@ __global__ void __launch_bounds__(kGateThreads) gate_pass1(const __nv_bfloat16* 
   }
 }
 
-__global__ void __launch_bounds__(1024) gate_pass2(const double* __restrict__ partials, int nparts, float threshold,
-                                                   float* __restrict__ rel_out, int32_t* __restrict__ skip_out) {
-  __shared__ double sn[1024], sd[1024];
+// The per-CTA partials combined in a fixed tree order (one 1024-thread CTA);
+// the totals land in sn[0], sd[0].
+__device__ __forceinline__ void combine_partials(const double* __restrict__ partials, int nparts, double* sn,
+                                                 double* sd) {
   double tn = 0.0, td = 0.0;
   for (int k = threadIdx.x; k < nparts; k += blockDim.x) {
     tn += partials[2 * k];
@@ -114,16 +115,41 @@ __global__ void __launch_bounds__(1024) gate_pass2(const double* __restrict__ pa
     }
     __syncthreads();
   }
+}
+
+// rel = num / den (0 when both are 0, +inf when only den is), skip = rel < threshold.
+__device__ __forceinline__ void decide(double num, double den, float threshold, float* rel_out, int32_t* skip_out) {
+  double rel;
+  if (den == 0.0)
+    rel = (num == 0.0) ? 0.0 : __longlong_as_double(0x7ff0000000000000ll);  // +inf
+  else
+    rel = num / den;
+  rel_out[0] = static_cast<float>(rel);
+  skip_out[0] = (rel < static_cast<double>(threshold)) ? 1 : 0;
+}
+
+__global__ void __launch_bounds__(1024) gate_pass2(const double* __restrict__ partials, int nparts, float threshold,
+                                                   float* __restrict__ rel_out, int32_t* __restrict__ skip_out) {
+  __shared__ double sn[1024], sd[1024];
+  combine_partials(partials, nparts, sn, sd);
+  if (threadIdx.x == 0) decide(sn[0], sd[0], threshold, rel_out, skip_out);
+}
+
+// Sharded form: the shard's totals (sum |a - b|, sum |b|) in fp64, to be summed
+// across ranks before gate_finalize decides.
+__global__ void __launch_bounds__(1024) gate_pass2_sums(const double* __restrict__ partials, int nparts,
+                                                        double* __restrict__ sums_out) {
+  __shared__ double sn[1024], sd[1024];
+  combine_partials(partials, nparts, sn, sd);
   if (threadIdx.x == 0) {
-    const double num = sn[0], den = sd[0];
-    double rel;
-    if (den == 0.0)
-      rel = (num == 0.0) ? 0.0 : __longlong_as_double(0x7ff0000000000000ll);  // +inf
-    else
-      rel = num / den;
-    rel_out[0] = static_cast<float>(rel);
-    skip_out[0] = (rel < static_cast<double>(threshold)) ? 1 : 0;
+    sums_out[0] = sn[0];
+    sums_out[1] = sd[0];
   }
+}
+
+__global__ void gate_finalize(const double* __restrict__ sums, float threshold, float* __restrict__ rel_out,
+                              int32_t* __restrict__ skip_out) {
+  if (threadIdx.x == 0) decide(sums[0], sums[1], threshold, rel_out, skip_out);
 }
 
 cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold, float* rel_out, int32_t* skip_out,
@@ -134,6 +160,23 @@ cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   gate_pass2<<<1, 1024, 0, stream>>>(partials, g, threshold, rel_out, skip_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* sums_out, double* partials,
+                             cudaStream_t stream) {
+  const int g = gate_num_ctas(n);
+  gate_pass1<<<g, kGateThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(a),
+                                             static_cast<const __nv_bfloat16*>(b), n, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gate_pass2_sums<<<1, 1024, 0, stream>>>(partials, g, sums_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
+                                 cudaStream_t stream) {
+  gate_finalize<<<1, 32, 0, stream>>>(sums, threshold, rel_out, skip_out);
   return cudaGetLastError();
 }
 

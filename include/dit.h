@@ -180,6 +180,20 @@ DIT_API size_t fbcache_gate_workspace_bytes(int64_t n);
 DIT_API dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float threshold, float* rel_out,
                         int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream);
 
+/* The gate over a residual split across ranks (sequence-parallel runs): each
+ * rank computes its shard's totals, sums_out[0] = sum |r_cur - r_prev| and
+ * sums_out[1] = sum |r_prev| (fp64, device, 8-byte aligned; same kernels and
+ * order as fbcache_gate); the caller adds the totals across ranks (an
+ * all-reduce of two doubles) and fbcache_gate_finalize decides.  Every rank
+ * then holds the same rel and skip.  Workspace as fbcache_gate. */
+DIT_API dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int64_t n, double* sums_out,
+                                     void* workspace, size_t workspace_bytes, dit_stream_t stream);
+
+/* rel = sums[0] / sums[1] (0 when both are 0, +inf when only sums[1] is),
+ * skip = rel < threshold, written to rel_out / skip_out (device). */
+DIT_API dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
+                                         dit_stream_t stream);
+
 /* fbcache_gate without a workspace argument (the pages have no counterpart:
  * this is a convenience of this library).  For callers that cannot give the
  * library device memory, e.g. a plug-in run by a host framework that owns the

@@ -156,3 +156,20 @@ def test_gate_last_computed_policy_matches_oracle():
             ref = t
     assert got == [s for _, s in ref_dec]
     assert dit.read_error() == 0
+
+
+def test_gate_sums_and_finalize_reproduce_the_gate():
+    """fbcache_gate_sums + fbcache_gate_finalize on the whole tensor give fbcache_gate's
+    rel bit for bit; from two shards' totals added together, the same decision."""
+    for eps in (1e-2, 0.3):
+        cur, prev = synth.gate_pair(4608, 3072 // 4, eps, device=DEV)
+        rel, skip = dit.fbcache_gate(cur, prev, 0.12)
+        rel2, skip2 = dit.fbcache_gate_finalize(dit.fbcache_gate_sums(cur, prev), 0.12)
+        assert torch.equal(rel, rel2) and torch.equal(skip, skip2)
+        h = cur.shape[0] // 2
+        tot = dit.fbcache_gate_sums(cur[:h], prev[:h]) + dit.fbcache_gate_sums(cur[h:], prev[h:])
+        rel3, skip3 = dit.fbcache_gate_finalize(tot, 0.12)
+        ref = G.relative_l1(cur.cpu(), prev.cpu())
+        assert abs(rel3.item() - ref) <= 1e-6 * ref
+        assert int(skip3.item()) == int(G.skip(ref, 0.12))
+    assert dit.read_error() == 0

@@ -51,6 +51,8 @@ def test_entry_points_report_unsupported_without_an_sm100_device():
     assert L.dit_rope_tables(A16, 16, 16, 24, 24, 1e4, A16, A16, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate(A16, A16, 64, 0.1, A16, A16, A16, 1 << 20, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate_noalloc(A16, A16, 64, 0.1, A16, A16, None) == DIT_ERR_UNSUPPORTED
+    assert L.fbcache_gate_sums(A16, A16, 64, A16, A16, 1 << 20, None) == DIT_ERR_UNSUPPORTED
+    assert L.fbcache_gate_finalize(A16, 0.1, A16, A16, None) == DIT_ERR_UNSUPPORTED
     assert L.dit_selftest_wait_timeout(None) == DIT_ERR_UNSUPPORTED
     assert L.dit_read_error(None) == DIT_ERR_UNSUPPORTED
 
