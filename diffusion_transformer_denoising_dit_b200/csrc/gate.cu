@@ -11,7 +11,9 @@
 // HBM-bound: 4 bytes read per element, ~3 flops.  Pass 1 streams both inputs
 // with 16-byte loads (4 per input in flight per thread) over up to 1184 CTAs, fp32 per-thread partials,
 // fp64 per-CTA combine; pass 2 (one CTA) combines the CTA partials in a fixed
-// tree order, so the result is deterministic for a given n.
+// tree order, so the result is deterministic for a given n.  For a residual split
+// across ranks, gate_pass2_sums stops at the two totals (summed across ranks by
+// the caller) and gate_finalize takes the decision from the summed totals.
 #include <cuda_bf16.h>
 
 #include <mutex>
