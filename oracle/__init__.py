@@ -26,6 +26,8 @@ open is stated where it is used.
 Parity status: attention, RoPE, the e4m3 quantiser and the gate are pinned by
 closed forms, invariants, brute force and independent library special cases
 (tests/test_oracle_*.py).  ``fp8.simulated_attention`` is a diagnostic of our
-own reading of an unspecified quantised scheme: parity unpinned.
+own reading of an unspecified quantised scheme: the reading cannot be pinned to
+the pages, its implementation is pinned by closed forms and invariants of that
+reading (and planted mistakes fail them).
 """
 from . import attention, fp8, gate, rope  # noqa: F401

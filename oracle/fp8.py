@@ -21,10 +21,16 @@ scaling; the readings used here:
   divided by the row sum of the unquantised P.
 
 ``simulated_attention`` follows those steps in fp64 on quantised operands.
-It is a diagnostic of our own reading (parity unpinned): it separates the
-quantisation floor from kernel errors.  Its row max is the exact one, where a
-streaming kernel uses a running max, so it matches a kernel only to within
-the quantisation noise.
+The scheme is our reading (the pages define none), so it is a diagnostic: it
+separates the quantisation floor from kernel errors.  Its implementation of
+that reading is pinned by closed forms and invariants (tests): Q = 0 gives the
+mean of the dequantised V (with unequal V block scales), one-hot scores give
+one dequantised V row, permuting whole K/V blocks changes nothing, V * 2^k
+scales O exactly, and a Q block scaled by 2^k equals its rows at 2^k sigma;
+each of a list of planted mistakes (a misindexed block scale, the per-head V
+maximum replaced, the row sum taken over quantised P, sigma dropped) fails one
+of them.  Its row max is the exact one, where a streaming kernel uses a
+running max, so it matches a kernel only to within the quantisation noise.
 """
 from __future__ import annotations
 
@@ -91,7 +97,7 @@ def smooth_k(k: np.ndarray) -> np.ndarray:
 
 def simulated_attention(q, k, v, scale=None, pos=None, axes=None, theta=10000.0,
                         q_block=128, kv_block=64, smooth=True, rows=None):
-    """fp64 attention on e4m3-quantised operands (diagnostic; parity unpinned)."""
+    """fp64 attention on e4m3-quantised operands (diagnostic of our FP8 reading)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     if pos is not None:
         q = _rope.apply(q, pos, axes, theta)

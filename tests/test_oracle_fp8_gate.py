@@ -186,3 +186,80 @@ def test_policy_last_computed_on_the_drift_trace():
 def test_policy_rejects_unknown_name():
     with pytest.raises(ValueError):
         gate.trace_decisions([np.ones(3)], 0.1, policy="nope")
+
+
+# --- simulated_attention: closed forms and invariants of the FP8 reading -------------
+
+
+def _dequant_rows(v, block=64):
+    """V as the FP8 scheme sees it: e4m3 codes times their block scale."""
+    codes, sc = fp8.quantize_blocks(v, block)
+    return codes * np.repeat(sc, block, axis=-1)[..., : v.shape[-2], None]
+
+
+def test_simulated_q_zero_gives_the_mean_of_dequantised_v():
+    """Q = 0: every score is 0 and p = 1.  The second V block's scale is half the
+    first's, so its P is 448 * 0.5 = 224, still exact in e4m3, and O is the plain
+    mean of the dequantised V: P * v8 * sV_max / 448 = sV(j) * v8."""
+    rng = np.random.default_rng(11)
+    v = rng.uniform(-1.0, 1.0, size=(1, 1, 128, 16))
+    v[0, 0, 3, 5] = 4.0       # block 0 amax 4
+    v[0, 0, 70, 2] = -2.0     # block 1 amax 2: half the scale
+    q = np.zeros_like(v)
+    k = rng.standard_normal(v.shape)
+    o = fp8.simulated_attention(q, k, v, smooth=False)
+    want = _dequant_rows(v).mean(axis=-2, keepdims=True)
+    np.testing.assert_allclose(o, np.broadcast_to(want, o.shape), rtol=0, atol=1e-14)
+
+
+def test_simulated_one_hot_scores_give_one_dequantised_row():
+    """K = a I, Q rows = b e_pi(i) with sigma a b = 40: exp(-40) * 448 quantises to 0,
+    so each output row is the dequantised V row of its partner key."""
+    d, n = 64, 64
+    a, b = 64.0, 40.0
+    k = (a * np.eye(d))[None, None]
+    perm = np.random.default_rng(12).permutation(n)
+    q = (b * np.eye(d)[perm])[None, None]
+    v = np.random.default_rng(13).standard_normal((1, 1, n, d))
+    sigma = 40.0 / (a * b)
+    o = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False)
+    want = _dequant_rows(v)[:, :, perm]
+    np.testing.assert_allclose(o, want, rtol=1e-14, atol=1e-14)
+
+
+def test_simulated_is_invariant_to_permuting_whole_kv_blocks():
+    """Moving whole 64-key blocks of K and V together moves their scales with them."""
+    rng = np.random.default_rng(14)
+    q, k, v = (rng.standard_normal((1, 2, 256, 32)) for _ in range(3))
+    k[..., 5] *= 8.0
+    q[..., 5] *= 8.0
+    order = [2, 0, 3, 1]
+    idx = np.concatenate([np.arange(64 * b, 64 * (b + 1)) for b in order])
+    o = fp8.simulated_attention(q, k, v)
+    o2 = fp8.simulated_attention(q, k[:, :, idx], v[:, :, idx])
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+
+
+def test_simulated_scales_exactly_with_powers_of_two():
+    """V * 4 scales every V block scale by 4 with the same codes: O * 4 exactly; Q * 2
+    with sigma / 2 leaves every score unchanged: the same O exactly."""
+    rng = np.random.default_rng(15)
+    q, k, v = (rng.standard_normal((1, 1, 192, 32)) for _ in range(3))
+    o = fp8.simulated_attention(q, k, v, scale=0.2)
+    assert np.array_equal(fp8.simulated_attention(q, k, 4.0 * v, scale=0.2), 4.0 * o)
+    assert np.array_equal(fp8.simulated_attention(2.0 * q, k, v, scale=0.1), o)
+
+
+def test_simulated_q_block_scales_follow_their_rows():
+    """Scaling the rows of the second 128-token Q block by 4 scales only that block's
+    Q scale (same codes): its rows equal those computed with 4 sigma, the first
+    block's rows do not move."""
+    rng = np.random.default_rng(16)
+    q, k, v = (rng.standard_normal((1, 1, 256, 32)) for _ in range(3))
+    q2 = q.copy()
+    q2[:, :, 128:] *= 4.0
+    o = fp8.simulated_attention(q, k, v, scale=0.1)
+    o2 = fp8.simulated_attention(q2, k, v, scale=0.1)
+    o4 = fp8.simulated_attention(q, k, v, scale=0.4)
+    assert np.array_equal(o2[:, :, :128], o[:, :, :128])
+    assert np.array_equal(o2[:, :, 128:], o4[:, :, 128:])
