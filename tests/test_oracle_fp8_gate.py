@@ -189,6 +189,8 @@ def test_policy_rejects_unknown_name():
 
 
 # --- simulated_attention: closed forms and invariants of the FP8 reading -------------
+# Each pin takes the implementation as an argument, so that the planted-mistake test
+# below can run the same pins against mutated copies of the oracle.
 
 
 def _dequant_rows(v, block=64):
@@ -197,7 +199,7 @@ def _dequant_rows(v, block=64):
     return codes * np.repeat(sc, block, axis=-1)[..., : v.shape[-2], None]
 
 
-def test_simulated_q_zero_gives_the_mean_of_dequantised_v():
+def _pin_q_zero(sim):
     """Q = 0: every score is 0 and p = 1.  The second V block's scale is half the
     first's, so its P is 448 * 0.5 = 224, still exact in e4m3, and O is the plain
     mean of the dequantised V: P * v8 * sV_max / 448 = sV(j) * v8."""
@@ -207,12 +209,12 @@ def test_simulated_q_zero_gives_the_mean_of_dequantised_v():
     v[0, 0, 70, 2] = -2.0     # block 1 amax 2: half the scale
     q = np.zeros_like(v)
     k = rng.standard_normal(v.shape)
-    o = fp8.simulated_attention(q, k, v, smooth=False)
+    o = sim(q, k, v, smooth=False)
     want = _dequant_rows(v).mean(axis=-2, keepdims=True)
     np.testing.assert_allclose(o, np.broadcast_to(want, o.shape), rtol=0, atol=1e-14)
 
 
-def test_simulated_one_hot_scores_give_one_dequantised_row():
+def _pin_one_hot(sim):
     """K = a I, Q rows = b e_pi(i) with sigma a b = 40: exp(-40) * 448 quantises to 0,
     so each output row is the dequantised V row of its partner key."""
     d, n = 64, 64
@@ -221,36 +223,31 @@ def test_simulated_one_hot_scores_give_one_dequantised_row():
     perm = np.random.default_rng(12).permutation(n)
     q = (b * np.eye(d)[perm])[None, None]
     v = np.random.default_rng(13).standard_normal((1, 1, n, d))
-    sigma = 40.0 / (a * b)
-    o = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False)
-    want = _dequant_rows(v)[:, :, perm]
-    np.testing.assert_allclose(o, want, rtol=1e-14, atol=1e-14)
+    o = sim(q, k, v, scale=40.0 / (a * b), smooth=False)
+    np.testing.assert_allclose(o, _dequant_rows(v)[:, :, perm], rtol=1e-14, atol=1e-14)
 
 
-def test_simulated_is_invariant_to_permuting_whole_kv_blocks():
+def _pin_block_permutation(sim):
     """Moving whole 64-key blocks of K and V together moves their scales with them."""
     rng = np.random.default_rng(14)
     q, k, v = (rng.standard_normal((1, 2, 256, 32)) for _ in range(3))
     k[..., 5] *= 8.0
     q[..., 5] *= 8.0
-    order = [2, 0, 3, 1]
-    idx = np.concatenate([np.arange(64 * b, 64 * (b + 1)) for b in order])
-    o = fp8.simulated_attention(q, k, v)
-    o2 = fp8.simulated_attention(q, k[:, :, idx], v[:, :, idx])
-    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+    idx = np.concatenate([np.arange(64 * b, 64 * (b + 1)) for b in (2, 0, 3, 1)])
+    np.testing.assert_allclose(sim(q, k[:, :, idx], v[:, :, idx]), sim(q, k, v), rtol=1e-12, atol=1e-12)
 
 
-def test_simulated_scales_exactly_with_powers_of_two():
+def _pin_powers_of_two(sim):
     """V * 4 scales every V block scale by 4 with the same codes: O * 4 exactly; Q * 2
     with sigma / 2 leaves every score unchanged: the same O exactly."""
     rng = np.random.default_rng(15)
     q, k, v = (rng.standard_normal((1, 1, 192, 32)) for _ in range(3))
-    o = fp8.simulated_attention(q, k, v, scale=0.2)
-    assert np.array_equal(fp8.simulated_attention(q, k, 4.0 * v, scale=0.2), 4.0 * o)
-    assert np.array_equal(fp8.simulated_attention(2.0 * q, k, v, scale=0.1), o)
+    o = sim(q, k, v, scale=0.2)
+    assert np.array_equal(sim(q, k, 4.0 * v, scale=0.2), 4.0 * o)
+    assert np.array_equal(sim(2.0 * q, k, v, scale=0.1), o)
 
 
-def test_simulated_q_block_scales_follow_their_rows():
+def _pin_q_blocks(sim):
     """Scaling the rows of the second 128-token Q block by 4 scales only that block's
     Q scale (same codes): its rows equal those computed with 4 sigma, the first
     block's rows do not move."""
@@ -258,8 +255,48 @@ def test_simulated_q_block_scales_follow_their_rows():
     q, k, v = (rng.standard_normal((1, 1, 256, 32)) for _ in range(3))
     q2 = q.copy()
     q2[:, :, 128:] *= 4.0
-    o = fp8.simulated_attention(q, k, v, scale=0.1)
-    o2 = fp8.simulated_attention(q2, k, v, scale=0.1)
-    o4 = fp8.simulated_attention(q, k, v, scale=0.4)
+    o = sim(q, k, v, scale=0.1)
+    o2 = sim(q2, k, v, scale=0.1)
+    o4 = sim(q, k, v, scale=0.4)
     assert np.array_equal(o2[:, :, :128], o[:, :, :128])
     assert np.array_equal(o2[:, :, 128:], o4[:, :, 128:])
+
+
+_SIM_PINS = [_pin_q_zero, _pin_one_hot, _pin_block_permutation, _pin_powers_of_two, _pin_q_blocks]
+
+
+@pytest.mark.parametrize("pin", _SIM_PINS, ids=lambda f: f.__name__[5:])
+def test_simulated_attention_pins(pin):
+    pin(fp8.simulated_attention)
+
+
+# plausible mistakes, planted in a copy of the oracle's own source (CPU only)
+_SIM_MUTATIONS = {
+    "per_head_v_max_replaced": ("* (svmax / E4M3_MAX) / l", "* (svc.mean() / E4M3_MAX) / l"),
+    "row_sum_over_quantised_p": ("/ l\n", "/ (p8.sum(axis=1, keepdims=True) * 2.0)\n"),
+    "kv_block_scale_misindexed": ("svc = np.repeat(sv[b, h], kv_block)[:N]",
+                                  "svc = np.roll(np.repeat(sv[b, h], kv_block)[:N], 1)"),
+    "q_block_scale_misindexed": ("sqr = np.repeat(sq[b, h], q_block)[:N]",
+                                 "sqr = np.roll(np.repeat(sq[b, h], q_block)[:N], q_block)"),
+    "sigma_dropped": ("s = sigma * (q8", "s = 1.0 * (q8"),
+    "v_scale_not_folded_into_p": ("quantize_e4m3(p * (E4M3_MAX * svc / svmax)[None, :])",
+                                  "quantize_e4m3(p * E4M3_MAX)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_SIM_MUTATIONS))
+def test_simulated_attention_pins_catch_planted_mistakes(name):
+    import inspect
+    old, new = _SIM_MUTATIONS[name]
+    src = inspect.getsource(fp8.simulated_attention)
+    assert old in src, name
+    ns = dict(vars(fp8))
+    exec(src.replace(old, new, 1), ns)
+    mutant = ns["simulated_attention"]
+    failed = 0
+    for pin in _SIM_PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            failed += 1
+    assert failed >= 1, name
