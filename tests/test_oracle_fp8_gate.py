@@ -70,6 +70,24 @@ def test_block_scales_put_block_amax_on_448():
     assert fp8.block_scales(z, 64)[0, 0, 0] == 1.0
 
 
+def test_block_quantisation_within_e4m3_error_bound():
+    """Blocks six orders of magnitude apart, each with a planted amax: every scale is
+    that amax / 448 exactly, and every dequantised element is within e4m3's rounding
+    error of the input (half a step: 2^-4 |x| in the normal range, 2^-10 scale below
+    it).  A scale taken from a neighbouring block saturates or underflows there."""
+    x = rng.uniform(-1.0, 1.0, size=(1, 2, 300, 16))
+    mags = np.array([1e3, 1e-3, 1e3, 1e-3, 1.0])
+    amax = mags * 1.5
+    for b in range(5):
+        x[..., 64 * b:64 * (b + 1), :] *= mags[b]
+        x[..., 64 * b + 7, 3] = -amax[b]
+    codes, sc = fp8.quantize_blocks(x, 64)
+    np.testing.assert_array_equal(sc, np.broadcast_to(amax / 448.0, sc.shape))
+    rep = np.repeat(amax / 448.0, 64)[:300][None, None, :, None]
+    err = np.abs(codes * rep - x)
+    assert np.all(err <= 2.0 ** -4 * np.abs(x) + 2.0 ** -10 * rep)
+
+
 def test_smoothing_leaves_exact_attention_unchanged():
     q, k, v = (rng.standard_normal((1, 2, 80, 32)) for _ in range(3))
     k = k + 5.0

@@ -1,0 +1,143 @@
+"""Planted mistakes in the rotary-embedding, e4m3 and cache-gate oracles (no GPU).
+
+Each case builds a copy of one oracle module with one plausible mistake
+planted in its source (a flipped sign, a wrong index, a dropped term, a
+different rounding rule, a non-strict comparison ...), swaps the copy in for
+the real module inside that module's committed pin tests, runs them, and
+requires at least one pin to fail.  The real oracle modules are never
+modified.
+"""
+import inspect
+import types
+
+import pytest
+
+import test_oracle_fp8_gate as T8
+import test_oracle_rope as TR
+from oracle import fp8, gate, rope
+
+
+def _mutant(module, edits):
+    """A fresh module object holding module's source with each (old, new) edit applied once."""
+    src = inspect.getsource(module)
+    for old, new in edits:
+        assert old in src, old
+        src = src.replace(old, new, 1)
+    m = types.ModuleType(module.__name__ + "_planted")
+    m.__package__ = module.__package__
+    exec(compile(src, f"<planted {module.__name__}>", "exec"), m.__dict__)
+    return m
+
+
+def _count_failing(pins):
+    failed = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+ROPE_PINS = [
+    TR.test_golden_hand_values,
+    TR.test_matches_complex_multiplication,
+    TR.test_pair_norms_preserved,
+    TR.test_position_zero_is_identity,
+    TR.test_inverse_rotation,
+    lambda: TR.test_scores_depend_only_on_relative_position((2, 9, 4)),
+    TR.test_axes_are_independent,
+    TR.test_angles_table_layout,
+]
+
+ROPE_MISTAKES = {
+    "rotation_direction_reversed": [("x0 * c - x1 * s", "x0 * c + x1 * s"),
+                                    ("x0 * s + x1 * c", "-x0 * s + x1 * c")],
+    "one_sine_sign_flipped": [("x0 * c - x1 * s", "x0 * c + x1 * s")],
+    "frequency_over_whole_head": [("-2.0 * p / da", "-2.0 * p / d")],
+    "frequency_exponent_halved": [("-2.0 * p / da", "-1.0 * p / da")],
+    "rotate_half_pairs": [("x0 = x[..., 0::2]", "x0 = x[..., : x.shape[-1] // 2]"),
+                          ("x1 = x[..., 1::2]", "x1 = x[..., x.shape[-1] // 2:]"),
+                          ("y[..., 0::2] =", "y[..., : x.shape[-1] // 2] ="),
+                          ("y[..., 1::2] =", "y[..., x.shape[-1] // 2:] =")],
+    "every_axis_uses_axis_0_position": [("pos[:, a] * freq", "pos[:, 0] * freq")],
+    "pair_offset_dropped": [("out[:, off // 2 + p]", "out[:, p]")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(ROPE_MISTAKES))
+def test_rope_pins_catch_planted_mistakes(name, monkeypatch):
+    monkeypatch.setattr(TR, "rope", _mutant(rope, ROPE_MISTAKES[name]))
+    assert _count_failing(ROPE_PINS) >= 1, name
+
+
+E4M3_PINS = [
+    T8.test_code_table_round_trip,
+    T8.test_ties_round_to_even_mantissa,
+    T8.test_golden_e4m3,
+    T8.test_matches_torch_float8_cast,
+    T8.test_saturation,
+    T8.test_block_scales_put_block_amax_on_448,
+    T8.test_block_quantisation_within_e4m3_error_bound,
+    T8.test_smoothing_leaves_exact_attention_unchanged,
+]
+
+E4M3_MISTAKES = {
+    "ties_away_from_zero": [("np.round(ax / quantum)", "np.floor(ax / quantum + 0.5)")],
+    "no_saturation": [("r = np.minimum(r, E4M3_MAX)", "r = r")],
+    "subnormal_floor_one_binade_low": [("_MIN_NORMAL_EXP = -6", "_MIN_NORMAL_EXP = -7")],
+    "two_mantissa_bits": [("_MANT_BITS = 3", "_MANT_BITS = 2")],
+    "block_amax_mapped_to_240": [("a / E4M3_MAX, 1.0", "a / 240.0, 1.0")],
+    "zero_block_scale_zero": [("a / E4M3_MAX, 1.0", "a / E4M3_MAX, 0.0")],
+    "block_scales_shifted": [("rep = np.repeat(sc, block, axis=-1)[..., : x.shape[-2]]",
+                              "rep = np.roll(np.repeat(sc, block, axis=-1)[..., : x.shape[-2]], 1, axis=-1)")],
+    "smoothing_mean_over_channels": [("k.mean(axis=-2, keepdims=True)", "k.mean(axis=-1, keepdims=True)")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(E4M3_MISTAKES))
+def test_e4m3_pins_catch_planted_mistakes(name, monkeypatch):
+    monkeypatch.setattr(T8, "fp8", _mutant(fp8, E4M3_MISTAKES[name]))
+    assert _count_failing(E4M3_PINS) >= 1, name
+
+
+GATE_PINS = [
+    T8.test_golden_gate,
+    T8.test_gate_brute_force_on_tiny_sweep,
+    T8.test_gate_zero_denominator,
+    T8.test_gate_strict_threshold,
+    T8.test_gate_symmetric_scaling,
+    T8.test_trace_decisions_follow_drift,
+    T8.test_policy_consecutive_on_geometric_growth,
+    T8.test_policy_last_computed_accumulates_until_threshold,
+    T8.test_policy_warmup_forces_early_steps,
+    T8.test_policy_last_computed_on_the_drift_trace,
+]
+
+GATE_MISTAKES = {
+    "denominator_from_current_step": [("den = float(np.abs(b).sum())", "den = float(np.abs(a).sum())")],
+    "squared_difference": [("num = float(np.abs(a - b).sum())", "num = float(((a - b) ** 2).sum())")],
+    "threshold_not_strict": [("return rel < threshold", "return rel <= threshold")],
+    "zero_denominator_always_inf": [('return 0.0 if num == 0.0 else float("inf")', 'return float("inf")')],
+    "reference_never_moves": [("        if not s:\n            ref = t", "        if not s:\n            pass")],
+    "reference_always_moves": [("        if not s:\n            ref = t", "        ref = t")],
+    "warmup_off_by_one": [("and t >= warmup", "and t > warmup")],
+    "policies_swapped": [('base = t - 1 if policy == "consecutive" else ref',
+                          'base = ref if policy == "consecutive" else t - 1')],
+}
+
+
+@pytest.mark.parametrize("name", sorted(GATE_MISTAKES))
+def test_gate_pins_catch_planted_mistakes(name, monkeypatch):
+    monkeypatch.setattr(T8, "gate", _mutant(gate, GATE_MISTAKES[name]))
+    assert _count_failing(GATE_PINS) >= 1, name
+
+
+def test_unmutated_copies_pass_every_pin(monkeypatch):
+    """The harness itself: copies built with no edit pass every pin."""
+    monkeypatch.setattr(TR, "rope", _mutant(rope, []))
+    monkeypatch.setattr(T8, "fp8", _mutant(fp8, []))
+    monkeypatch.setattr(T8, "gate", _mutant(gate, []))
+    assert _count_failing(ROPE_PINS) == 0
+    assert _count_failing(E4M3_PINS) == 0
+    assert _count_failing(GATE_PINS) == 0
