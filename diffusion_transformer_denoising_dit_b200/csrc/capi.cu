@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -27,7 +28,7 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode{nullptr};  // set once, read by make_map
 
 // Per-device set-up on first use: architecture check and the error word's address.
 const DeviceState* device_state() {
@@ -45,17 +46,18 @@ const DeviceState* device_state() {
     if (!s.err) s.sm100 = false;
     s.probed = true;
   }
-  if (!g_encode) {
+  if (!g_encode.load()) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      g_encode.store(reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn));
   }
   return &s;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Element strides must keep every row 16-byte aligned for TMA / vector access.
 bool strides_ok(const int64_t s[3], int elem_bytes) {
@@ -64,11 +66,18 @@ bool strides_ok(const int64_t s[3], int elem_bytes) {
   return true;
 }
 
+// Every dimension of extent > 1 advances (a positive stride: neither TMA nor the
+// kernels broadcast), and token rows do not overlap (token stride >= d).
+bool layout_ok(const int64_t s[3], int B, int H, int N, int d) {
+  return !(B > 1 && s[0] <= 0) && !(H > 1 && s[1] <= 0) && !(N > 1 && s[2] < d);
+}
+
 // 4-D tiled tensor map over [B][H][N][d] with the given element strides;
 // box = {box_inner elements, box_rows tokens, 1, 1}, 128-byte swizzle.
 bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, int B, int H, int N, int d,
               const int64_t s[3], int box_inner, int box_rows) {
-  if (!g_encode) return false;
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = g_encode.load();
+  if (!encode) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(B)};
   // A size-1 dimension never advances; give it a harmless legal stride.
@@ -79,7 +88,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const vo
                            static_cast<cuuint64_t>(bs * elem_bytes)};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = encode(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -134,6 +143,7 @@ dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, do
   if (d0 < 0 || d1 < 0 || d2 < 0 || (d0 | d1 | d2) & 1 || d0 + d1 + d2 < 2 || d0 + d1 + d2 > 256)
     return DIT_ERR_INVALID_ARG;
   if (!(theta > 0.0) || !std::isfinite(theta)) return DIT_ERR_INVALID_ARG;
+  if (!aligned4(pos) || !aligned4(cos_out) || !aligned4(sin_out)) return DIT_ERR_ALIGNMENT;
   const DeviceState* ds = device_state();
   if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
   return launch_status(dit::launch_rope_tables(pos, N, d0, d1, d2, theta, cos_out, sin_out,
@@ -149,6 +159,8 @@ dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d, const 
   if (!aligned16(x) || !aligned16(y) || !strides_ok(sx, 2) || !strides_ok(sy, dtype ? 4 : 2) ||
       !valid_rope_tables(cos_tab, sin_tab))
     return DIT_ERR_ALIGNMENT;
+  if (!layout_ok(sx, B, H, N, d) || !layout_ok(sy, B, H, N, d)) return DIT_ERR_INVALID_ARG;
+  if (x == y && (sx[0] != sy[0] || sx[1] != sy[1] || sx[2] != sy[2])) return DIT_ERR_INVALID_ARG;  // in place
   const DeviceState* ds = device_state();
   if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
   dit::RopeJob job;
@@ -180,12 +192,15 @@ dit_status attn_bf16_impl(const void* q, const void* k, const void* v, void* o, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !strides_ok(sq, 2) || !strides_ok(sk, 2) ||
       !strides_ok(sv, 2) || !strides_ok(so, 2) || !valid_rope_tables(rope_cos, rope_sin))
     return DIT_ERR_ALIGNMENT;
+  if (!layout_ok(sq, B, H, N, d) || !layout_ok(sk, B, H, N, d) || !layout_ok(sv, B, H, N, d) ||
+      !layout_ok(so, B, H, N, d) || o == q || o == k || o == v)
+    return DIT_ERR_INVALID_ARG;
   const bool rope = rope_cos != nullptr;
   const size_t need = dit_attn_bf16_workspace_bytes(B, H, N, d, rope);
   if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
     return DIT_ERR_WORKSPACE;
   const DeviceState* ds = device_state();
-  if (!ds || !ds->sm100 || !g_encode) return DIT_ERR_UNSUPPORTED;
+  if (!ds || !ds->sm100 || !g_encode.load()) return DIT_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   const void* ka = k;
@@ -267,11 +282,14 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !strides_ok(sq, 2) || !strides_ok(sk, 2) ||
       !strides_ok(sv, 2) || !strides_ok(so, 2) || !valid_rope_tables(rope_cos, rope_sin))
     return DIT_ERR_ALIGNMENT;
+  if (!layout_ok(sq, B, H, N, d) || !layout_ok(sk, B, H, N, d) || !layout_ok(sv, B, H, N, d) ||
+      !layout_ok(so, B, H, N, d) || o == q || o == k || o == v)
+    return DIT_ERR_INVALID_ARG;
   const size_t need = dit_attn_fp8_workspace_bytes(B, H, N, d, q_block, kv_block);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return DIT_ERR_WORKSPACE;
   const DeviceState* ds = device_state();
-  if (!ds || !ds->sm100 || !g_encode) return DIT_ERR_UNSUPPORTED;
+  if (!ds || !ds->sm100 || !g_encode.load()) return DIT_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   dit::Fp8Prep p;
@@ -324,7 +342,7 @@ dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float 
                         int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream) {
   if (!r_cur || !r_prev || !rel_out || !skip_out || n < 1) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
-  if (!aligned16(r_cur) || !aligned16(r_prev)) return DIT_ERR_ALIGNMENT;
+  if (!aligned16(r_cur) || !aligned16(r_prev) || !aligned4(rel_out) || !aligned4(skip_out)) return DIT_ERR_ALIGNMENT;
   const size_t need = fbcache_gate_workspace_bytes(n);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 7u)) return DIT_ERR_WORKSPACE;
   const DeviceState* ds = device_state();
@@ -349,7 +367,7 @@ dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel
                                  dit_stream_t stream) {
   if (!sums || !rel_out || !skip_out) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(sums) & 7u) return DIT_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(sums) & 7u) || !aligned4(rel_out) || !aligned4(skip_out)) return DIT_ERR_ALIGNMENT;
   const DeviceState* ds = device_state();
   if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
   return launch_status(dit::launch_gate_finalize(sums, threshold, rel_out, skip_out,

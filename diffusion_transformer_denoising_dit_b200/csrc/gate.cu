@@ -237,7 +237,8 @@ extern "C" DIT_API dit_status fbcache_gate_noalloc(const void* r_cur, const void
                                                    float* rel_out, int32_t* skip_out, dit_stream_t stream) {
   if (!r_cur || !r_prev || !rel_out || !skip_out || n < 1) return DIT_ERR_INVALID_ARG;
   if (!(threshold == threshold) || threshold > 3.4e38f || threshold < -3.4e38f) return DIT_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(r_cur) & 15u) || (reinterpret_cast<uintptr_t>(r_prev) & 15u))
+  if ((reinterpret_cast<uintptr_t>(r_cur) & 15u) || (reinterpret_cast<uintptr_t>(r_prev) & 15u) ||
+      (reinterpret_cast<uintptr_t>(rel_out) & 3u) || (reinterpret_cast<uintptr_t>(skip_out) & 3u))
     return DIT_ERR_ALIGNMENT;
   // the fixed array must hold every pass-1 partial for this n
   if (2 * static_cast<int64_t>(dit::gate_num_ctas(n)) > kNoAllocScratchDoubles) return DIT_ERR_WORKSPACE;

@@ -42,6 +42,10 @@
  *   - Tensors [B,H,N,d] are described by element strides {batch, head,
  *     token}; the channel dimension is contiguous.  Strides and base pointers
  *     must be 16-byte aligned (a TMA requirement): bf16 strides multiple of 8.
+ *     A dimension of extent > 1 needs a positive stride (broadcast views are
+ *     not supported) and token rows may not overlap (token stride >= d when
+ *     N > 1); DIT_ERR_INVALID_ARG otherwise.  Layouts such as [B,N,H,d]
+ *     (head stride d, token stride H*d) are fine.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
  *   - A non-DIT_OK return means nothing was enqueued.  Failures inside a
  *     kernel (a bounded wait that ran out) are recorded in a device error
@@ -98,12 +102,15 @@ DIT_API dit_status dit_selftest_wait_timeout(dit_stream_t stream);
 
 /* Builds cos/sin tables, fp32 [N][d/2] each, d = d0+d1+d2, from int32
  * position ids pos[N][3] (device).  Angles are formed and evaluated in fp64
- * and rounded once to fp32.  d0,d1,d2 even and >= 0, d <= 256, N >= 1. */
+ * and rounded once to fp32.  d0,d1,d2 even and >= 0, d <= 256, N >= 1;
+ * pos, cos_out, sin_out 4-byte aligned (the attention kernels read the tables
+ * 16 bytes at a time, so allocate them 16-byte aligned). */
 DIT_API dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, double theta, float* cos_out,
                            float* sin_out, dit_stream_t stream);
 
 /* y = rotary(x) for x, y [B,H,N,d] with element strides sx/sy {batch, head,
- * token}; y may alias x exactly (in place).  dtype: 0 = bf16 in and out,
+ * token}; y may alias x exactly (in place, with sy equal to sx; a partial
+ * overlap is not detected and is the caller's error).  dtype: 0 = bf16 in and out,
  * 1 = bf16 in, fp32 out.  Math in fp32, output rounded once (RNE).
  * d in {64, 128}; tables as built by dit_rope_tables. */
 DIT_API dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d, const int64_t sx[3], const int64_t sy[3],
@@ -121,7 +128,8 @@ DIT_API size_t dit_attn_bf16_workspace_bytes(int B, int H, int N, int d, int has
 
 /* O = attention(Q, K, V) in BF16 with fp32 accumulation and softmax.
  * q, k, v: bf16 [B,H,N,d] inputs; o: bf16 [B,H,N,d] output (must not alias
- * q, k or v).  rope_cos/rope_sin: tables [N][d/2] or both NULL (no rotary).
+ * q, k or v: o equal to one of them is DIT_ERR_INVALID_ARG; a partial
+ * overlap is not detected).  rope_cos/rope_sin: tables [N][d/2] or both NULL (no rotary).
  * softmax_scale <= 0 selects 1/sqrt(d).  d in {64, 128}; N >= 1.
  * workspace: device buffer of at least dit_attn_bf16_workspace_bytes, 256-byte
  * aligned (may be NULL when that size is 0). */
@@ -176,7 +184,7 @@ DIT_API size_t fbcache_gate_workspace_bytes(int64_t n);
  * elements (fp32 per-thread partials, fp64 combine in a fixed order, so the
  * result is deterministic); skip_out[0] = (rel < threshold).  rel_out and
  * skip_out are device pointers; read skip_out on the host to branch.
- * n >= 1; r_cur, r_prev 16-byte aligned. */
+ * n >= 1; r_cur, r_prev 16-byte aligned; rel_out, skip_out 4-byte aligned. */
 DIT_API dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float threshold, float* rel_out,
                         int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream);
 

@@ -39,7 +39,7 @@ S = B._i64x3
 A16 = 1 << 20          # a fake 16-byte aligned device address (never dereferenced)
 
 
-def _attn(L, q=A16, k=A16, v=A16, o=A16, Bn=1, H=1, N=16, d=64, s=(1024, 1024, 64), cos=None, sin=None,
+def _attn(L, q=A16, k=A16, v=A16, o=A16 + 4096, Bn=1, H=1, N=16, d=64, s=(1024, 1024, 64), cos=None, sin=None,
           scale=0.0, ws=None, wsb=0):
     st = S(*s)
     return L.dit_attn_bf16(q, k, v, o, Bn, H, N, d, st, st, st, st, cos, sin, scale, ws, wsb, None)
@@ -60,6 +60,43 @@ def test_attention_argument_validation():
     assert L.dit_attn_bf16_workspace_bytes(1, 1, 16, 64, 0) == 0
 
 
+def test_layout_validation_rejects_broadcast_and_overlap():
+    """A dimension of extent > 1 must advance and token rows may not overlap; a
+    zero stride on an extent-1 dimension is harmless."""
+    L = B.lib()
+    assert _attn(L, H=2, s=(1 << 20, 0, 64)) == 1       # heads broadcast
+    assert _attn(L, Bn=2, s=(0, 1024, 64)) == 1         # batch broadcast
+    assert _attn(L, s=(1024, 1024, 0)) == 1             # every token the same row
+    assert _attn(L, s=(1024, 1024, 32)) == 1            # rows overlap (token stride < d)
+    # legal layouts get past the layout check to the workspace check (no device call)
+    assert _attn(L, s=(0, 0, 64), cos=A16, sin=A16) == 4                   # B = H = 1
+    assert _attn(L, H=4, s=(16 * 4 * 64, 64, 4 * 64), cos=A16, sin=A16) == 4  # [B, N, H, d]
+
+
+def test_output_may_not_be_an_input():
+    L = B.lib()
+    for name in ("q", "k", "v"):
+        assert _attn(L, **{name: A16 + 4096}, o=A16 + 4096) == 1
+    st = S(1 << 20, 1 << 20, 128)
+    args = (A16, A16, A16, A16, 1, 1, 1024, 128, st, st, st, st, None, None, 0.0, 128, 64, 1, A16, 1 << 30, None)
+    assert L.dit_attn_fp8(*args) == 1                    # o == q
+
+
+def test_rope_apply_in_place_needs_equal_strides():
+    L = B.lib()
+    a, b = S(4096, 4096, 64), S(8192, 4096, 64)
+    assert L.rope_apply(A16, A16, 2, 1, 64, 64, a, b, A16, A16, 0, None) == 1
+
+
+def test_small_outputs_alignment():
+    L = B.lib()
+    assert L.fbcache_gate(A16, A16, 100, 0.1, A16 + 2, A16, A16, 1 << 20, None) == 3    # rel_out
+    assert L.fbcache_gate(A16, A16, 100, 0.1, A16, A16 + 1, A16, 1 << 20, None) == 3    # skip_out
+    assert L.fbcache_gate_noalloc(A16, A16, 100, 0.1, A16 + 2, A16, None) == 3
+    assert L.fbcache_gate_finalize(A16, 0.1, A16, A16 + 2, None) == 3
+    assert L.dit_rope_tables(A16 + 2, 10, 16, 24, 24, 1e4, A16, A16, None) == 3        # pos
+
+
 def test_skippable_attention_argument_validation():
     L = B.lib()
     st = S(1024, 1024, 64)
@@ -71,7 +108,7 @@ def test_skippable_attention_argument_validation():
 def test_fp8_argument_validation():
     L = B.lib()
     st = S(1024 * 128, 1024 * 128, 128)
-    args = (A16, A16, A16, A16, 1, 1, 1024, 128, st, st, st, st, None, None, 0.0)
+    args = (A16, A16, A16, A16 + 4096, 1, 1, 1024, 128, st, st, st, st, None, None, 0.0)
     assert L.dit_attn_fp8(*args, 64, 64, 1, A16, 1 << 30, None) == 2      # q_block != 128
     assert L.dit_attn_fp8(*args, 128, 64, 1, None, 0, None) == 4          # no workspace
     small = L.dit_attn_fp8_workspace_bytes(1, 1, 1024, 128, 128, 64) - 1
