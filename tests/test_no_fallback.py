@@ -41,10 +41,11 @@ def test_entry_points_report_unsupported_without_an_sm100_device():
     L = B.lib()
     st = B._i64x3(1024, 1024, 64)
     st8 = B._i64x3(16 * 128, 16 * 128, 128)
-    args = (A16, A16, A16, A16, 1, 1, 16, 64, st, st, st, st, None, None, 0.0)
+    O = A16 + (1 << 16)  # the output may not be an input
+    args = (A16, A16, A16, O, 1, 1, 16, 64, st, st, st, st, None, None, 0.0)
     assert L.dit_attn_bf16(*args, None, 0, None) == DIT_ERR_UNSUPPORTED
     assert L.dit_attn_bf16_skippable(*args, None, 0, A16, None) == DIT_ERR_UNSUPPORTED
-    args8 = (A16, A16, A16, A16, 1, 1, 16, 128, st8, st8, st8, st8, None, None, 0.0)
+    args8 = (A16, A16, A16, O, 1, 1, 16, 128, st8, st8, st8, st8, None, None, 0.0)
     need = L.dit_attn_fp8_workspace_bytes(1, 1, 16, 128, 128, 64)
     assert L.dit_attn_fp8(*args8, 128, 64, 1, A16, need, None) == DIT_ERR_UNSUPPORTED
     assert L.rope_apply(A16, A16, 1, 1, 16, 64, st, st, A16, A16, 0, None) == DIT_ERR_UNSUPPORTED
