@@ -105,9 +105,33 @@ def _strides(t: torch.Tensor):
 
 
 def _need_cuda(*ts):
+    devs = set()
     for t in ts:
         if t is not None and not t.is_cuda:
             raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+        if t is not None:
+            devs.add(t.device)
+    if len(devs) > 1:
+        raise ValueError(f"all tensors must be on one device, got {sorted(map(str, devs))}")
+
+
+def _check_tables(cos, sin, N: int, d: int):
+    """The kernels read rotary tables as fp32 [N, d/2] rows, 16 bytes at a time."""
+    if (cos is None) != (sin is None):
+        raise ValueError("pass both rotary tables or neither")
+    for t in (cos, sin):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (N, d // 2) or not t.is_contiguous()):
+            raise ValueError(f"rotary tables must be contiguous float32 [{N}, {d // 2}] (as rope_tables builds them)")
+
+
+def _check_out(out, shape, dtype):
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype:
+        raise ValueError(f"out must be {dtype} of shape {list(shape)}, got {out.dtype} {list(out.shape)}")
+
+
+def _check_bytes(buf, name: str):
+    if buf is not None and not buf.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
 
 
 def read_error(stream=None) -> int:
@@ -141,12 +165,18 @@ def rope_tables(pos: torch.Tensor, axes, theta: float = 10000.0):
 
 def rope_apply(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, out_dtype=torch.bfloat16, out=None):
     """Rotary embedding of x [B,H,N,d] (bf16) -> bf16 or fp32 (out may be x for in-place bf16)."""
-    _need_cuda(x, cos, sin)
+    _need_cuda(x, cos, sin, out)
     if x.dtype != torch.bfloat16:
         raise ValueError("x must be bf16")
     B, H, N, d = x.shape
+    _check_tables(cos, sin, N, d)
+    if cos is None:
+        raise ValueError("rope_apply needs the rotary tables")
     if out is None:
         out = torch.empty(B, H, N, d, device=x.device, dtype=out_dtype)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or float32")
+    _check_out(out, x.shape, out.dtype)
     dt = {torch.bfloat16: 0, torch.float32: 1}[out.dtype]
     _check("rope_apply", lib().rope_apply(x.data_ptr(), out.data_ptr(), B, H, N, d, _strides(x), _strides(out),
                                           cos.data_ptr(), sin.data_ptr(), dt, _stream(x)))
@@ -161,7 +191,7 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
     skip (BF16 only): a device int32 flag, e.g. FBCacheGate's output; when it is
     non-zero at the time the kernels run, the call does nothing and ``out`` keeps
     its previous contents."""
-    _need_cuda(q, k, v, cos, sin, skip)
+    _need_cuda(q, k, v, cos, sin, skip, out, workspace)
     if skip is not None and (precision != "bf16" or skip.dtype != torch.int32 or skip.numel() < 1):
         raise ValueError("skip must be a CUDA int32 flag and is supported for precision='bf16'")
     for t in (q, k, v):
@@ -170,8 +200,11 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
     if not (q.shape == k.shape == v.shape):
         raise ValueError("q, k, v must have the same [B, H, N, d] shape")
     B, H, N, d = q.shape
+    _check_tables(cos, sin, N, d)
+    _check_bytes(workspace, "workspace")
     if out is None:
         out = torch.empty(B, H, N, d, device=q.device, dtype=torch.bfloat16)
+    _check_out(out, q.shape, torch.bfloat16)
     sc = 0.0 if scale is None else float(scale)
     L = lib()
     if precision == "bf16":
@@ -231,9 +264,18 @@ def fp8_workspace_views(ws: torch.Tensor, B: int, H: int, N: int, d: int = 128, 
     return out
 
 
+def _check_flags(rel_out, skip_out):
+    if rel_out is not None and (rel_out.dtype != torch.float32 or rel_out.numel() < 1):
+        raise ValueError("rel_out must be a float32 tensor of at least one element")
+    if skip_out is not None and (skip_out.dtype != torch.int32 or skip_out.numel() < 1):
+        raise ValueError("skip_out must be an int32 tensor of at least one element")
+
+
 def fbcache_gate(r_cur, r_prev, threshold: float, rel_out=None, skip_out=None, workspace=None):
     """(rel fp32 [1], skip int32 [1]) device tensors for two bf16 residuals of equal size."""
-    _need_cuda(r_cur, r_prev)
+    _need_cuda(r_cur, r_prev, rel_out, skip_out, workspace)
+    _check_flags(rel_out, skip_out)
+    _check_bytes(workspace, "workspace")
     if r_cur.dtype != torch.bfloat16 or r_prev.dtype != torch.bfloat16:
         raise ValueError("residuals must be bf16")
     if r_cur.numel() != r_prev.numel() or not r_cur.is_contiguous() or not r_prev.is_contiguous():
@@ -255,7 +297,11 @@ def fbcache_gate(r_cur, r_prev, threshold: float, rel_out=None, skip_out=None, w
 
 def fbcache_gate_sums(r_cur, r_prev, sums_out=None, workspace=None):
     """Shard totals (sum |r_cur - r_prev|, sum |r_prev|) as a device float64 [2] tensor."""
-    _need_cuda(r_cur, r_prev)
+    _need_cuda(r_cur, r_prev, sums_out, workspace)
+    _check_bytes(workspace, "workspace")
+    if sums_out is not None and (sums_out.dtype != torch.float64 or sums_out.numel() < 2
+                                 or not sums_out.is_contiguous()):
+        raise ValueError("sums_out must be a contiguous float64 tensor of at least two elements")
     if r_cur.dtype != torch.bfloat16 or r_prev.dtype != torch.bfloat16 or r_cur.shape != r_prev.shape:
         raise ValueError("r_cur, r_prev must be bf16 tensors of one shape")
     r_cur, r_prev = r_cur.contiguous(), r_prev.contiguous()
@@ -274,7 +320,8 @@ def fbcache_gate_sums(r_cur, r_prev, sums_out=None, workspace=None):
 
 def fbcache_gate_finalize(sums, threshold: float, rel_out=None, skip_out=None):
     """(rel, skip) device tensors from totals summed across shards."""
-    _need_cuda(sums)
+    _need_cuda(sums, rel_out, skip_out)
+    _check_flags(rel_out, skip_out)
     if sums.dtype != torch.float64 or sums.numel() < 2:
         raise ValueError("sums must be a device float64 [2] tensor")
     if rel_out is None:

@@ -188,3 +188,21 @@ def test_gate_flag_drives_skippable_attention_without_host_reads():
         else:
             assert torch.equal(out, ref)
     assert dit.read_error() == 0
+
+
+def test_binding_rejects_bad_tables_and_outputs_before_launch():
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w, device=DEV)
+    pos = synth.positions(w.T, w.G)
+    cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    with pytest.raises(ValueError):
+        dit.attention(q, k, v, cos[:-1], sin[:-1])                      # a table shorter than N
+    with pytest.raises(ValueError):
+        dit.attention(q, k, v, cos.bfloat16(), sin.bfloat16())          # wrong table dtype
+    with pytest.raises(ValueError):
+        dit.attention(q, k, v, cos, None)                               # one table only
+    with pytest.raises(ValueError):
+        dit.attention(q, k, v, cos, sin, out=torch.empty(q.shape, device=DEV, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        dit.rope_apply(q, cos[:-1], sin[:-1])
+    assert dit.read_error() == 0

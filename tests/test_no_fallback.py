@@ -64,3 +64,21 @@ def test_binding_does_not_import_the_oracle():
     importlib.reload(B)
     importlib.reload(dit)
     assert not any(m == "oracle" or m.startswith("oracle.") for m in sys.modules)
+
+
+def test_binding_metadata_checks():
+    """What the C ABI cannot see (table lengths, dtypes, devices) is checked before any call."""
+    c = torch.zeros(10, 32)
+    B._check_tables(None, None, 10, 64)
+    B._check_tables(c, c, 10, 64)
+    for bad in ((c, None), (c[:9], c[:9]), (c.double(), c.double()), (c.t().contiguous().t(), c)):
+        with pytest.raises(ValueError):
+            B._check_tables(*bad, 10, 64)
+    with pytest.raises(ValueError):
+        B._check_out(torch.zeros(1, 2, 10, 64), (1, 2, 10, 64), torch.bfloat16)
+    with pytest.raises(ValueError):
+        B._check_flags(torch.zeros(1, dtype=torch.float64), None)
+    with pytest.raises(ValueError):
+        B._check_flags(None, torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        B._check_bytes(torch.zeros(4, 4, dtype=torch.uint8).t(), "workspace")
