@@ -203,31 +203,29 @@ dit_status attn_bf16_impl(const void* q, const void* k, const void* v, void* o, 
   if (!ds || !ds->sm100 || !g_encode.load()) return DIT_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  const void* ka = k;
-  int64_t ska[3] = {sk[0], sk[1], sk[2]};
-  if (rope) {
-    // K is rotated once per head into the workspace (every CTA of the head reads
-    // each K tile); Q is rotated by the attention kernel as it loads each Q tile.
-    void* kr = workspace;
-    const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
-    dit::RopeJob job;
-    job.x = k;
-    job.y = kr;
-    for (int i = 0; i < 3; ++i) {
-      job.sx[i] = sk[i];
-      job.sy[i] = cs[i];
-    }
-    cudaError_t e = dit::launch_rope_apply(&job, 1, B, H, N, d, rope_cos, rope_sin, 0, st, skip);
-    if (e != cudaSuccess) return DIT_ERR_LAUNCH;
-    ka = kr;
-    for (int i = 0; i < 3; ++i) ska[i] = cs[i];
-  }
+  // K is rotated once per head into the workspace (every CTA of the head reads
+  // each K tile); Q is rotated by the attention kernel as it loads each Q tile.
+  const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
+  const void* ka = rope ? workspace : k;
+  const int64_t* ska = rope ? cs : sk;
+  // Every map is built before the first launch, so an error return leaves nothing enqueued.
   CUtensorMap tq, tk, tv;
   // Q tiles are 128 tokens, K/V tiles kAttnBlockN tokens; boxes are 128 bytes wide.
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, B, H, N, d, sq, 64, 128) ||
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ka, B, H, N, d, ska, 64, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, B, H, N, d, sv, 64, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
+  if (rope) {
+    dit::RopeJob job;
+    job.x = k;
+    job.y = workspace;
+    for (int i = 0; i < 3; ++i) {
+      job.sx[i] = sk[i];
+      job.sy[i] = cs[i];
+    }
+    cudaError_t e = dit::launch_rope_apply(&job, 1, B, H, N, d, rope_cos, rope_sin, 0, st, skip);
+    if (e != cudaSuccess) return DIT_ERR_LAUNCH;
+  }
   dit::AttnOut out{};  // value-initialised: every pointer not set below is null
   out.o = o;
   for (int i = 0; i < 3; ++i) out.so[i] = so[i];
@@ -279,6 +277,7 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return DIT_ERR_INVALID_ARG;
   if (d != 128 || q_block != 128 || kv_block != 64) return DIT_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H > 65535) return DIT_ERR_UNSUPPORTED;  // the prologue's grid.y is B*H
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !strides_ok(sq, 2) || !strides_ok(sk, 2) ||
       !strides_ok(sv, 2) || !strides_ok(so, 2) || !valid_rope_tables(rope_cos, rope_sin))
     return DIT_ERR_ALIGNMENT;
@@ -313,14 +312,15 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   p.v_scale_max = reinterpret_cast<float*>(w); w += align256(bh * 4);
   p.k_partial = reinterpret_cast<float*>(w);
 
-  if (dit::launch_fp8_prologue(p, st) != cudaSuccess) return DIT_ERR_LAUNCH;
   const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
+  // Every map is built before the first launch, so an error return leaves nothing enqueued.
   CUtensorMap tq, tk, tv;
   // e4m3: one 128-byte row holds all d = 128 channels of a token.
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.q8, B, H, N, d, cs, 128, 128) ||
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.k8, B, H, N, d, cs, 128, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.v8, B, H, N, d, cs, 128, dit::kAttnBlockN))
     return DIT_ERR_ALIGNMENT;
+  if (dit::launch_fp8_prologue(p, st) != cudaSuccess) return DIT_ERR_LAUNCH;
   dit::AttnOut out{};  // value-initialised: every pointer not set below is null
   out.o = o;
   for (int i = 0; i < 3; ++i) out.so[i] = so[i];

@@ -110,6 +110,7 @@ cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int 
   a.skip = skip;
   const int64_t total = static_cast<int64_t>(B) * H * N * (d / 8);
   const int64_t blocks = (total + 255) / 256;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;  // grid.x limit; nothing launched
   dim3 grid(static_cast<unsigned>(blocks), njobs);
   rope_apply_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();

@@ -166,8 +166,8 @@ DIT_API size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_bl
  * quantised to e4m3 (RNE, saturating) with one fp32 scale amax/448 per block
  * of q_block (Q) or kv_block (K, V) tokens.  Scores accumulate in fp32; P is
  * e4m3 with the V block scale folded in; the row sum uses the fp32 P.
- * Supported: d = 128, q_block = 128, kv_block = 64.  Arguments otherwise as
- * dit_attn_bf16. */
+ * Supported: d = 128, q_block = 128, kv_block = 64, B * H <= 65535
+ * (DIT_ERR_UNSUPPORTED otherwise).  Arguments otherwise as dit_attn_bf16. */
 DIT_API dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
                         const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,

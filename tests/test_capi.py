@@ -113,6 +113,9 @@ def test_fp8_argument_validation():
     assert L.dit_attn_fp8(*args, 128, 64, 1, None, 0, None) == 4          # no workspace
     small = L.dit_attn_fp8_workspace_bytes(1, 1, 1024, 128, 128, 64) - 1
     assert L.dit_attn_fp8(*args, 128, 64, 1, A16, small, None) == 4
+    big = S(40000 * 1024 * 128, 1024 * 128, 128)
+    wide = (A16, A16, A16, A16 + 4096, 2, 40000, 1024, 128, big, big, big, big, None, None, 0.0)
+    assert L.dit_attn_fp8(*wide, 128, 64, 1, None, 0, None) == 2          # B * H > 65535 (before the workspace)
 
 
 def test_gate_and_rope_validation():
