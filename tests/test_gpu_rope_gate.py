@@ -39,6 +39,20 @@ def test_rope_apply_fp32_within_1e3(name):
     assert err <= 1e-4 * max(1.0, np.abs(ref).max())   # what fp32 math actually gives
 
 
+def test_rope_apply_bench_configuration_sampled_heads():
+    """The 2048-px workload at full size (24 heads x 16896 tokens, the bench's K pass in
+    fp32 output): every token of the first and last head against the oracle."""
+    w = synth.WORKLOADS["flux2k"]
+    pos = synth.positions(w.T, w.G)
+    q, _, _ = synth.qkv(w, device=DEV)
+    c, s = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    y = dit.rope_apply(q, c, s, out_dtype=torch.float32)
+    for h in (0, w.H - 1):
+        ref = R.apply(q[:, h].cpu().double().numpy(), pos.numpy(), w.axes, w.theta)
+        err = np.abs(y[:, h].cpu().double().numpy() - ref).max()
+        assert err <= 1e-3, (h, err)
+
+
 def test_rope_apply_bf16_within_one_ulp_and_in_place():
     w = synth.WORKLOADS["tiny"]
     pos = synth.positions(w.T, w.G)
@@ -120,6 +134,16 @@ def test_gate_degenerate_cases():
     prev = torch.tensor([1.0, -2.0, 0.5, 4.0, 8.0] * 20, dtype=torch.bfloat16)
     assert _gate(prev * 1.125, prev, 0.2) == (0.125, 1)
     assert _gate(-prev, prev, 0.2) == (2.0, 0)
+
+
+def test_gate_bench_configuration():
+    """The bench's residual pair at full size (16896 x 3072 bf16, 51.9 M elements),
+    called as the bench calls it, against the fp64 oracle."""
+    r_prev, r_cur = synth.gate_pair(16896, 3072, 0.05, seed=4000, device=DEV)
+    rel, skip = _gate(r_cur, r_prev, 0.12)
+    ref = G.relative_l1(r_cur.cpu(), r_prev.cpu())
+    assert abs(rel - ref) <= 1e-5 * ref
+    assert abs(ref - 0.12) > 1e-4 and skip == int(G.skip(ref, 0.12))
 
 
 def test_gate_is_deterministic():
