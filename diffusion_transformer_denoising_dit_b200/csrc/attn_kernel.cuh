@@ -17,7 +17,10 @@
 //   warp 9     MMA issuer (one thread) and TMEM owner
 //   warps 10-11 idle (they complete the third warpgroup for the register re-split)
 // Registers: launched at 168 per thread; the third warpgroup drops to kRegsAux and
-// the softmax warpgroups rise to kRegsSoftmax (2*128*kRegsSoftmax + 128*kRegsAux <= 64K).
+// the softmax warpgroups rise to kRegsSoftmax.  setmaxnreg draws on the block's
+// launch registers, so 2*128*kRegsSoftmax + 128*kRegsAux (63,488) must not exceed
+// 384 * 168 = 64,512; the static_assert below only bounds it by the register file,
+// and a CPU test checks it against the count ptxas assigns.
 // BF16: RoPE of Q happens as Q is loaded: the softmax warpgroup that owns a Q
 // tile rotates the raw bf16 rows in shared memory with the cos/sin tables and
 // writes them back in place before the first MMA reads them.  K is rotated once
