@@ -50,7 +50,7 @@ def test_two_rank_max_over_ranks():
 
 
 def _ulysses_worker(rank, world, port, q):
-    """Two gloo ranks on CPU: the Ulysses exchanges around a CPU attention (the
+    """gloo ranks on CPU: the Ulysses exchanges around a CPU attention (the
     oracle's, injected; the library's own kernels need the GPU) and the sharded
     gate decision, against the unsharded results."""
     import datetime
@@ -84,7 +84,8 @@ def _ulysses_worker(rank, world, port, q):
         err = float(np.abs(o.numpy() - full[:, :, sl]).max())
         # sharded gate: shard totals, all-reduce, one decision everywhere
         cur, prev = synth.gate_pair(288, 128, 0.1)
-        rows = slice(rank * 144, (rank + 1) * 144)
+        m = 288 // world
+        rows = slice(rank * m, (rank + 1) * m)
 
         def sums(a, b):
             a64, b64 = a.double(), b.double()
@@ -102,21 +103,24 @@ def _ulysses_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.timeout(180)
-def test_two_rank_ulysses_exchange_and_sharded_gate():
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_exchange_and_sharded_gate(world):
+    """2 and 4 gloo ranks (4 heads: 2 or 1 per rank; 288 tokens: 144 or 72 per rank)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ulysses_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_ulysses_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = sorted(q.get(timeout=150) for _ in procs)
+    res = sorted(q.get(timeout=200) for _ in procs)
     for p in procs:
         p.join(timeout=30)
         assert p.exitcode == 0
+    assert [r[0] for r in res] == list(range(world))
     for rank, ok_layout, ok_round, err, rel, skip, ref_rel in res:
         assert ok_layout and ok_round
         assert err < 1e-12
         assert abs(rel - ref_rel) < 1e-12 * max(1.0, ref_rel)
         assert skip == (ref_rel < 0.12)
-    assert res[0][4] == res[1][4]  # both ranks hold the same rel
+    assert len({r[4] for r in res}) == 1  # every rank holds the same rel
