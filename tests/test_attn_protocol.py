@@ -29,6 +29,11 @@ stage an issued MMA still reads; the softmax reads S and writes P only while no
 issued MMA touches that half of the buffer; O is rescaled and read only while
 no PV into it is outstanding.  Planted protocol mistakes (negative controls)
 must each be caught.
+
+Faults: a load or an arrival can be made to never come; the bounded mbarrier
+waits then time out in every order the model can reach, and the tests record
+which losses end every role (the kernel reports DIT_ERR_TIMEOUT and exits) and
+which leave a role at a named barrier, which cannot time out.
 """
 import random
 
@@ -72,8 +77,17 @@ CONFIGS = {
 }
 
 
-def simulate(fp8, NK, NV, nkv, seed, mistake=None):
-    """Run one random interleaving; returns (errors, finished)."""
+def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
+    """Run one random interleaving; returns (errors, finished, timeouts).  With a
+    fault injected the result is already invalid once a wait has timed out, so
+    data hazards no longer stop the run and `errors` holds only a hang.
+
+    lost: a fault to inject -- ("load", kind, tile) for a TMA load that never
+    lands, or ("commit", barrier name, index, nth) for a commit arrival that
+    never comes.  Without a fault no wait may time out; with one, a role whose
+    bounded mbarrier wait cannot complete times out (returns false, as the
+    kernel's mbar_wait does after its limit) and takes the kernel's exit path.
+    """
     rng = random.Random(seed)
     split = pingpong = not fp8
     errors = []
@@ -85,6 +99,7 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
     v_empty = [MBar(2) for _ in range(NV)]
     s_full = [MBar(1), MBar(1)]
     pv_done = [MBar(1), MBar(1)]
+    bars = {"s_full": s_full, "pv_done": pv_done, "k_empty": k_empty, "v_empty": v_empty}
     p_ready = [Named(f"PReady{i}", 160, errors) for i in range(2)]
     p_half = [Named(f"PHalf{i}", 160, errors) for i in range(2)]
     turn = [Named(f"Turn{i}", 256, errors) for i in range(2)]
@@ -95,14 +110,23 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
     tma = []                            # loads in flight: (kind, slot, tile)
     queue, issued, completed = [], [0], [0]
     commits = []                        # (MMAs that must have completed, barrier)
+    commit_count = {}
 
     def fire_commits():
         while commits and commits[0][0] <= completed[0]:
             commits.pop(0)[1].arrive()
 
-    def commit(bar):
-        commits.append((issued[0], bar))
+    def commit(name, idx):
+        n = commit_count.get((name, idx), 0)
+        commit_count[(name, idx)] = n + 1
+        if lost == ("commit", name, idx, n):
+            return  # this arrival never comes
+        commits.append((issued[0], bars[name][idx]))
         fire_commits()
+
+    def load(kind, slot, tile):
+        if lost != ("load", kind, tile):
+            tma.append((kind, slot, tile))
 
     def issue(kind, i, tile, stage, halves):
         queue.append(dict(kind=kind, i=i, tile=tile, stage=stage, halves=halves))
@@ -110,6 +134,9 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
 
     def touching(i, half):
         return [m for m in queue if m["i"] == i and (m["kind"] == "S" or half in m["halves"])]
+
+    def pv_pending(i):
+        return any(m["kind"] == "PV" and m["i"] == i for m in queue)
 
     def complete_mma():
         m = queue.pop(0)
@@ -130,33 +157,38 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
         completed[0] += 1
         fire_commits()
 
-    def land(load):
-        tma.remove(load)
-        kind, slot, tile = load
+    def land(ld):
+        tma.remove(ld)
+        kind, slot, tile = ld
         if kind == "Q":
             qstate[slot] = "loaded"
             q_full[slot].arrive()
             return
-        stages, bars = (kstage, k_full) if kind == "K" else (vstage, v_full)
+        stages, full = (kstage, k_full) if kind == "K" else (vstage, v_full)
         mk = "S" if kind == "K" else "PV"
         if any(m["kind"] == mk and m["stage"] == slot for m in queue):
             errors.append(f"{kind} tile {tile} lands in stage {slot} while an issued MMA reads it")
         stages[slot] = tile
-        bars[slot].arrive()
+        full[slot].arrive()
 
     # ------------------------------------------------------------------ roles
+    # A role yields ("mbar", pred) for a bounded mbarrier wait (sent back True when
+    # it completes, False when it times out) or a bare predicate for a wait that
+    # cannot time out (named barriers) or a plain scheduling point.
     def producer():
         for i in range(2):
-            tma.append(("Q", i, 0))
+            load("Q", i, 0)
         for j in range(nkv):
             sk, sv = j % NK, j % NV
             if j >= NK:
                 par = ((j // NK) & 1) if mistake == "producer_parity_without_xor" else ((j // NK) & 1) ^ 1
-                yield lambda sk=sk, par=par: k_empty[sk].done(par)
-            tma.append(("K", sk, j))
+                if not (yield ("mbar", lambda sk=sk, par=par: k_empty[sk].done(par))):
+                    break
+            load("K", sk, j)
             if j >= NV:
-                yield lambda sv=sv, j=j: v_empty[sv].done(((j // NV) & 1) ^ 1)
-            tma.append(("V", sv, j))
+                if not (yield ("mbar", lambda sv=sv, j=j: v_empty[sv].done(((j // NV) & 1) ^ 1))):
+                    break
+            load("V", sv, j)
 
     def named_sync(bar, who, n):
         g = bar.gen
@@ -166,19 +198,25 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
     def mma():
         q_in = q_full if (fp8 or mistake == "mma_waits_unrotated_q") else q_ready
         halves_all = (0, 1)
-        yield lambda: q_in[0].done(0) and k_full[0].done(0)
-        issue("S", 0, 0, 0, halves_all)
-        commit(s_full[0])
-        commit(k_empty[0])
-        yield lambda: q_in[1].done(0)
-        issue("S", 1, 0, 0, halves_all)
-        commit(s_full[1])
-        commit(k_empty[0])
+        ok = (yield ("mbar", lambda: q_in[0].done(0))) and (yield ("mbar", lambda: k_full[0].done(0)))
+        if ok:
+            issue("S", 0, 0, 0, halves_all)
+            commit("s_full", 0)
+            commit("k_empty", 0)
+            ok = yield ("mbar", lambda: q_in[1].done(0))
+        if ok:
+            issue("S", 1, 0, 0, halves_all)
+            commit("s_full", 1)
+            commit("k_empty", 0)
         for j in range(1, nkv + 1):
+            if not ok:
+                break
             jj, sv, sk = j - 1, (j - 1) % NV, j % NK
-            yield lambda sv=sv, jj=jj: v_full[sv].done((jj // NV) & 1)
-            if j < nkv:
-                yield lambda sk=sk, j=j: k_full[sk].done((j // NK) & 1)
+            ok = yield ("mbar", lambda sv=sv, jj=jj: v_full[sv].done((jj // NV) & 1))
+            if ok and j < nkv:
+                ok = yield ("mbar", lambda sk=sk, j=j: k_full[sk].done((j // NK) & 1))
+            if not ok:
+                break
             for i in range(2):
                 early_s = mistake == "s_before_pv" and j < nkv
                 if early_s:
@@ -188,24 +226,27 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
                     issue("PV", i, jj, sv, (0,))
                 yield named_sync(p_ready[i], "mma", 32)
                 issue("PV", i, jj, sv, (1,) if split else halves_all)
-                commit(pv_done[i])
-                commit(v_empty[sv])
+                commit("pv_done", i)
+                commit("v_empty", sv)
                 if j < nkv and not early_s:
                     issue("S", i, j, sk, halves_all)
                 if j < nkv:
-                    commit(s_full[i])
-                    commit(k_empty[sk])
+                    commit("s_full", i)
+                    commit("k_empty", sk)
 
     def softmax(i):
         who = f"softmax{i}"
         if not fp8:
-            yield lambda: q_full[i].done(0)
-            if touching(i, 0):
-                errors.append(f"Q{i} rotated while an MMA reads it")
-            qstate[i] = "rotated"
-            q_ready[i].arrive()
+            if (yield ("mbar", lambda: q_full[i].done(0))):
+                if touching(i, 0):
+                    errors.append(f"Q{i} rotated while an MMA reads it")
+                qstate[i] = "rotated"
+            q_ready[i].arrive()  # arrives whether or not the tile came
+        ok = True
         for j in range(nkv):
-            yield lambda j=j: s_full[i].done(j & 1)
+            ok = yield ("mbar", lambda j=j: s_full[i].done(j & 1))
+            if not ok:
+                break
             if any(m["kind"] == "S" and m["i"] == i for m in queue) or buf[i] != [("S", j), ("S", j)]:
                 errors.append(f"softmax{i}({j}) reads S holding {buf[i]} with MMAs {len(queue)} in flight")
             grow = j > 0 and rng.random() < 0.5
@@ -219,9 +260,8 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
                     errors.append(f"softmax{i}({j}) writes P half {h} while an MMA touches it")
                 buf[i][h] = ("P", j)
                 if split and h == 0:
-                    if grow and mistake != "rescale_after_release":
-                        if any(m["kind"] == "PV" and m["i"] == i for m in queue):
-                            errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
+                    if grow and mistake != "rescale_after_release" and pv_pending(i):
+                        errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
                     p_half[i].arrive(who, 128)
                     yield lambda: True  # the MMA warp may run between the halves
             if pingpong:
@@ -229,43 +269,66 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
                     turn[1].arrive(who, 128)
                 elif j + 1 < nkv and mistake != "softmax0_skips_turn":
                     turn[0].arrive(who, 128)
-            if not split and grow and mistake != "rescale_after_release":
-                if any(m["kind"] == "PV" and m["i"] == i for m in queue):
-                    errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
+            if not split and grow and mistake != "rescale_after_release" and pv_pending(i):
+                errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
             p_ready[i].arrive(who, 128)
             if grow and mistake == "rescale_after_release":
                 yield lambda: True
-                if any(m["kind"] == "PV" and m["i"] == i for m in queue):
+                if pv_pending(i):
                     errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
-        yield lambda: pv_done[i].done((nkv - 1) & 1)
-        if any(m["kind"] == "PV" and m["i"] == i for m in queue):
+        if ok:
+            ok = yield ("mbar", lambda: pv_done[i].done((nkv - 1) & 1))
+        if ok and pv_pending(i):
             errors.append(f"softmax{i} reads O while a PV writes it")
 
     roles = {"producer": producer(), "mma": mma(), "softmax0": softmax(0), "softmax1": softmax(1)}
-    waiting = {name: (lambda: True) for name in roles}
+    waiting = {name: None for name in roles}   # None: about to start
     finished = set()
+    timeouts = []
+
+    def ready(name):
+        w = waiting[name]
+        if w is None:
+            return True
+        return (w[1] if isinstance(w, tuple) else w)()
+
+    def step(name, value):
+        try:
+            waiting[name] = roles[name].send(value)
+        except StopIteration:
+            finished.add(name)
+
+    hang = []
     for _ in range(100000):
-        if errors:
+        if errors and lost is None:
             break
-        options = [("role", n) for n in roles if n not in finished and waiting[n]()]
+        options = [("role", n) for n in roles if n not in finished and ready(n)]
         options += [("tma", ld) for ld in tma]
         if queue:
             options.append(("mma", None))
         if not options:
-            if len(finished) < len(roles):
-                errors.append("deadlock: " + ", ".join(sorted(set(roles) - finished)) + " blocked")
-            break
+            blocked = sorted(set(roles) - finished)
+            if not blocked:
+                break
+            bounded = [n for n in blocked if isinstance(waiting[n], tuple)]
+            if lost is None or not bounded:
+                hang.append(", ".join(blocked) + " blocked" + ("" if bounded else " on named barriers"))
+                errors.append(("deadlock: " if lost is None else "hang: ") + hang[-1])
+                break
+            name = rng.choice(bounded)
+            timeouts.append(name)
+            step(name, False)
+            continue
         kind, what = rng.choice(options)
         if kind == "tma":
             land(what)
         elif kind == "mma":
             complete_mma()
         else:
-            try:
-                waiting[what] = next(roles[what])
-            except StopIteration:
-                finished.add(what)
-    return errors, len(finished) == len(roles)
+            step(what, None if waiting[what] is None else True)
+    if lost is not None:
+        return hang, len(finished) == len(roles), timeouts
+    return errors, len(finished) == len(roles), timeouts
 
 
 @pytest.mark.parametrize("name", sorted(CONFIGS))
@@ -273,8 +336,8 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None):
 def test_protocol_completes_without_hazards(name, nkv):
     cfg = CONFIGS[name]
     for seed in range(400):
-        errors, finished = simulate(nkv=nkv, seed=seed, **cfg)
-        assert not errors and finished, (name, nkv, seed, errors[:3])
+        errors, finished, timeouts = simulate(nkv=nkv, seed=seed, **cfg)
+        assert not errors and finished and not timeouts, (name, nkv, seed, errors[:3])
 
 
 PLANTED = [
@@ -293,7 +356,56 @@ PLANTED = [
 def test_planted_protocol_mistakes_are_caught(mistake, name):
     cfg = CONFIGS[name]
     for seed in range(400):
-        errors, finished = simulate(nkv=7, seed=seed, mistake=mistake, **cfg)
+        errors, finished, _ = simulate(nkv=7, seed=seed, mistake=mistake, **cfg)
         if errors or not finished:
             return
     pytest.fail(f"{mistake} not caught in 400 interleavings")
+
+
+# Faults the bounded waits cover: a K or V load that never lands, a stage release
+# (tcgen05.commit on k_empty / v_empty) that never arrives, and in FP8 (where the
+# MMA warp itself waits for Q) a Q load that never lands.  Every role ends through
+# a wait that times out (the kernel records DIT_ERR_TIMEOUT) and the CTA reaches
+# its exit; none stays blocked on a named barrier.
+COVERED_FAULTS = [("load", "K", 0), ("load", "K", 2), ("load", "K", 5), ("load", "V", 0), ("load", "V", 3),
+                  ("commit", "k_empty", 0, 0), ("commit", "k_empty", 1, 1), ("commit", "v_empty", 0, 0),
+                  ("commit", "v_empty", 1, 1)]
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+@pytest.mark.parametrize("fault", COVERED_FAULTS, ids=lambda f: "-".join(map(str, f)))
+def test_lost_loads_and_releases_end_every_role(name, fault):
+    for seed in range(100):
+        hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=fault, **CONFIGS[name])
+        assert finished and not hang, (name, fault, seed, hang)
+        assert timeouts, (name, fault, seed)  # the loss is reported, not absorbed
+
+
+def test_lost_q_load_ends_every_role_in_fp8():
+    for seed in range(100):
+        hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=("load", "Q", 0), **CONFIGS["fp8_d128"])
+        assert finished and not hang and timeouts, (seed, hang)
+
+
+# Faults the bounded waits do not cover (named barriers cannot time out), found
+# by this model.  Both need a lost hardware arrival; the fault-free protocol
+# above never produces one.
+#  * s_full: if the tensor core's arrival is lost, the softmax warpgroup times out
+#    and leaves its loop without arriving at its P-ready named barrier, where the
+#    MMA warp then waits without a limit.
+#  * BF16 Q load: the softmax warpgroup that rotates Q arrives on q_ready even when
+#    its wait for the tile timed out, so the MMA warp may go on into the named
+#    barriers while the other warpgroup's wait times out (which timeout fires
+#    first decides).  Arriving on q_ready only when the tile came would close it.
+UNCOVERED_FAULTS = [(n, ("commit", "s_full", 0, 1)) for n in sorted(CONFIGS)] + \
+                   [(n, ("load", "Q", 0)) for n in ("bf16_d128", "bf16_d64")]
+
+
+@pytest.mark.parametrize("name,fault", UNCOVERED_FAULTS, ids=lambda x: x if isinstance(x, str) else "-".join(map(str, x)))
+def test_uncovered_faults_end_at_a_named_barrier(name, fault):
+    for seed in range(100):
+        hang, finished, _ = simulate(nkv=7, seed=seed, lost=fault, **CONFIGS[name])
+        if hang:
+            assert "mma" in hang[0] and "named barriers" in hang[0], hang
+            return
+    pytest.fail(f"{fault} ended every role in 100 interleavings")
