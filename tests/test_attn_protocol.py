@@ -77,10 +77,17 @@ CONFIGS = {
 }
 
 
-def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
+def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, report=None):
     """Run one random interleaving; returns (errors, finished, timeouts).  With a
     fault injected the result is already invalid once a wait has timed out, so
     data hazards no longer stop the run and `errors` holds only a hang.
+
+    fixes: the two failure-path changes planned for the kernel -- the rotating
+    warpgroup arrives on q_ready only when its Q tile came (and otherwise skips
+    its tile loop), and the producer waits, bounded, for the last load it issued
+    into every stage before it leaves.  A lost load is modelled as stalled: issued
+    and in flight, never landing.  report: a dict that receives the loads still in
+    flight when every role has ended and the stages whose drain wait gave up.
 
     lost: a fault to inject -- ("load", kind, tile) for a TMA load that never
     lands, or ("commit", barrier name, index, nth) for a commit arrival that
@@ -124,9 +131,13 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
         commits.append((issued[0], bars[name][idx]))
         fire_commits()
 
+    stalled = set()
+    drain_gave_up = set()
+
     def load(kind, slot, tile):
-        if lost != ("load", kind, tile):
-            tma.append((kind, slot, tile))
+        tma.append((kind, slot, tile))
+        if lost == ("load", kind, tile):
+            stalled.add((kind, slot, tile))  # issued, never lands
 
     def issue(kind, i, tile, stage, halves):
         queue.append(dict(kind=kind, i=i, tile=tile, stage=stage, halves=halves))
@@ -177,7 +188,8 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
     # cannot time out (named barriers) or a plain scheduling point.
     def producer():
         for i in range(2):
-            load("Q", i, 0)
+            load("Q", i, i)  # Q tile i (the tile index names which Q load a fault drops)
+        nk_issued = nv_issued = 0
         for j in range(nkv):
             sk, sv = j % NK, j % NV
             if j >= NK:
@@ -185,10 +197,22 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
                 if not (yield ("mbar", lambda sk=sk, par=par: k_empty[sk].done(par))):
                     break
             load("K", sk, j)
+            nk_issued += 1
             if j >= NV:
                 if not (yield ("mbar", lambda sv=sv, j=j: v_empty[sv].done(((j // NV) & 1) ^ 1))):
                     break
             load("V", sv, j)
+            nv_issued += 1
+        if fixes:  # drain: the last load issued into each stage has landed (phase index = tile // ring)
+            for i in range(2):
+                if not (yield ("mbar", lambda i=i: q_full[i].done(0))):
+                    drain_gave_up.add(("Q", i))
+            for kind, ring, issued_n, full in (("K", NK, nk_issued, k_full), ("V", NV, nv_issued, v_full)):
+                for st in range(min(ring, issued_n)):
+                    last = st + ((issued_n - 1 - st) // ring) * ring
+                    if not (yield ("mbar", lambda full=full, st=st, last=last, ring=ring:
+                                   full[st].done((last // ring) & 1))):
+                        drain_gave_up.add((kind, st))
 
     def named_sync(bar, who, n):
         g = bar.gen
@@ -236,14 +260,20 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
 
     def softmax(i):
         who = f"softmax{i}"
+        ok = True
         if not fp8:
-            if (yield ("mbar", lambda: q_full[i].done(0))):
+            q_ok = yield ("mbar", lambda: q_full[i].done(0))
+            if q_ok:
                 if touching(i, 0):
                     errors.append(f"Q{i} rotated while an MMA reads it")
                 qstate[i] = "rotated"
-            q_ready[i].arrive()  # arrives whether or not the tile came
-        ok = True
+            if q_ok or not fixes:
+                q_ready[i].arrive()  # the kernel today arrives whether or not the tile came
+            if fixes:
+                ok = q_ok
         for j in range(nkv):
+            if not ok:
+                break
             ok = yield ("mbar", lambda j=j: s_full[i].done(j & 1))
             if not ok:
                 break
@@ -303,13 +333,13 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
         if errors and lost is None:
             break
         options = [("role", n) for n in roles if n not in finished and ready(n)]
-        options += [("tma", ld) for ld in tma]
+        options += [("tma", ld) for ld in tma if ld not in stalled]
         if queue:
             options.append(("mma", None))
+        if len(finished) == len(roles):
+            break  # every role has ended: the CTA exits here
         if not options:
             blocked = sorted(set(roles) - finished)
-            if not blocked:
-                break
             bounded = [n for n in blocked if isinstance(waiting[n], tuple)]
             if lost is None or not bounded:
                 hang.append(", ".join(blocked) + " blocked" + ("" if bounded else " on named barriers"))
@@ -326,6 +356,9 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None):
             complete_mma()
         else:
             step(what, None if waiting[what] is None else True)
+    if report is not None:
+        report["in_flight_at_exit"] = list(tma)
+        report["drain_gave_up"] = set(drain_gave_up)
     if lost is not None:
         return hang, len(finished) == len(roles), timeouts
     return errors, len(finished) == len(roles), timeouts
@@ -409,3 +442,34 @@ def test_uncovered_faults_end_at_a_named_barrier(name, fault):
             assert "mma" in hang[0] and "named barriers" in hang[0], hang
             return
     pytest.fail(f"{fault} ended every role in 100 interleavings")
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_planned_failure_path_fixes(name):
+    """The planned changes, checked on the model before they go into the kernel:
+    fault-free runs stay free of hazards and of timeouts (so the drain's parity
+    formula is right) and end with nothing in flight; every load loss, Q included,
+    now ends every role; and a load still in flight when the roles end is always
+    one the drain waited for and gave up on."""
+    cfg = CONFIGS[name]
+    for nkv in (1, 2, 3, 5, 9):
+        for seed in range(150):
+            rep = {}
+            errors, finished, timeouts = simulate(nkv=nkv, seed=seed, fixes=True, report=rep, **cfg)
+            assert not errors and finished and not timeouts and not rep["in_flight_at_exit"], (nkv, seed, errors)
+    for fault in COVERED_FAULTS + [("load", "Q", 0), ("load", "Q", 1)]:
+        for seed in range(100):
+            rep = {}
+            hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=fault, fixes=True, report=rep, **cfg)
+            assert finished and not hang and timeouts, (fault, seed, hang)
+            for kind, slot, _ in rep["in_flight_at_exit"]:
+                assert (kind, slot) in rep["drain_gave_up"], (fault, seed, rep)
+
+
+def test_without_the_drain_a_stalled_load_is_left_behind_unwaited():
+    """Today's kernel: after a load stalls, the CTA ends with it in flight and no
+    wait for it (the planned drain waits for it, bounded, before leaving)."""
+    rep = {}
+    hang, finished, _ = simulate(nkv=7, seed=0, lost=("load", "K", 2), report=rep, **CONFIGS["bf16_d128"])
+    assert finished and not hang
+    assert ("K", 2 % 3, 2) in rep["in_flight_at_exit"] and not rep["drain_gave_up"]
