@@ -1,20 +1,21 @@
-"""Planted mistakes in the rotary-embedding, e4m3 and cache-gate oracles (no GPU).
+"""Planted mistakes in the attention, rotary-embedding, e4m3 and cache-gate oracles (no GPU).
 
 Each case builds a copy of one oracle module with one plausible mistake
 planted in its source (a flipped sign, a wrong index, a dropped term, a
 different rounding rule, a non-strict comparison ...), swaps the copy in for
 the real module inside that module's committed pin tests, runs them, and
-requires at least one pin to fail.  The real oracle modules are never
-modified.
+requires at least one pin to fail (an assertion, or an error a mutant raises).
+The real oracle modules are never modified.
 """
 import inspect
 import types
 
 import pytest
 
+import test_oracle_attention as TA
 import test_oracle_fp8_gate as T8
 import test_oracle_rope as TR
-from oracle import fp8, gate, rope
+from oracle import attention, fp8, gate, rope
 
 
 def _mutant(module, edits):
@@ -34,9 +35,48 @@ def _count_failing(pins):
     for pin in pins:
         try:
             pin()
-        except AssertionError:
+        except Exception:  # an assertion, or an error the mutant raises: the pin fails either way
             failed += 1
     return failed
+
+
+ATTENTION_PINS = [
+    TA.test_golden_hand_example,
+    TA.test_zero_q_gives_mean_v_with_and_without_rope,
+    TA.test_one_hot_scores_select_rows,
+    TA.test_permutation_equivariance,
+    TA.test_single_token_returns_v,
+    TA.test_constant_v_gives_constant_output,
+    TA.test_key_shift_invariance,
+    TA.test_matches_torch_sdpa_float64,
+    TA.test_brute_force_loops,
+    TA.test_row_subset_matches_full,
+    TA.test_rope_is_applied_to_q_and_k_not_v,
+    TA.test_round_bf16_matches_torch_cast_of_float32,
+    TA.test_round_bf16_ties_and_exact_values,
+    TA.test_bf16_operand_reading_is_rounded_rotation,
+]
+
+_SIGMA = "sigma = 1.0 / math.sqrt(d) if scale is None or scale <= 0 else float(scale)"
+ATTENTION_MISTAKES = {
+    "scale_argument_ignored": [(_SIGMA, "sigma = 1.0 / math.sqrt(d)")],
+    "default_scale_one": [(_SIGMA, "sigma = 1.0 if scale is None or scale <= 0 else float(scale)")],
+    "normalised_over_queries": [("/ e.sum(axis=1, keepdims=True)", "/ e.sum(axis=0, keepdims=True).T")],
+    "last_key_left_out_of_the_sum": [("/ e.sum(axis=1, keepdims=True)", "/ e[:, :-1].sum(axis=1, keepdims=True)")],
+    "v_rotated_too": [("    v = _f64(v)\n", "    v = rotate(v, pos, axes, theta)\n")],
+    "k_not_rotated": [("k = rotate(k, pos, axes, theta)", "k = _f64(k)")],
+    "bf16_operands_not_rounded": [("        q = round_bf16(q)\n        k = round_bf16(k)", "        q = q\n        k = k")],
+    "bf16_rounding_truncates": [("np.round(ax / q) * q", "np.floor(ax / q) * q")],
+    "bf16_one_bit_too_many": [("q = np.exp2(e - 7)", "q = np.exp2(e - 8)")],
+    "selected_rows_ignored": [("s = sigma * (q[b, h, sel] @ kt)", "s = sigma * (q[b, h, r0:r0 + len(sel)] @ kt)")],
+}
+
+
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")
+@pytest.mark.parametrize("name", sorted(ATTENTION_MISTAKES))
+def test_attention_pins_catch_planted_mistakes(name, monkeypatch):
+    monkeypatch.setattr(TA, "A", _mutant(attention, ATTENTION_MISTAKES[name]))
+    assert _count_failing(ATTENTION_PINS) >= 1, name
 
 
 ROPE_PINS = [
@@ -135,9 +175,11 @@ def test_gate_pins_catch_planted_mistakes(name, monkeypatch):
 
 def test_unmutated_copies_pass_every_pin(monkeypatch):
     """The harness itself: copies built with no edit pass every pin."""
+    monkeypatch.setattr(TA, "A", _mutant(attention, []))
     monkeypatch.setattr(TR, "rope", _mutant(rope, []))
     monkeypatch.setattr(T8, "fp8", _mutant(fp8, []))
     monkeypatch.setattr(T8, "gate", _mutant(gate, []))
+    assert _count_failing(ATTENTION_PINS) == 0
     assert _count_failing(ROPE_PINS) == 0
     assert _count_failing(E4M3_PINS) == 0
     assert _count_failing(GATE_PINS) == 0
