@@ -20,6 +20,13 @@ scaling; the readings used here:
   (P * 448 * sV(j) / sV_max), and the output is rescaled by sV_max / 448 and
   divided by the row sum of the unquantised P.
 
+An alternative reading of the Q.K^T step, SageAttention's (the quantised
+attention the ledger names): Q and K as per-block symmetric int8 (scale
+amax / 127, round to nearest even, clipped to +-127) with P.V still in e4m3;
+``simulated_attention(..., qk="int8")``.  Pinned by every code, ties, torch's
+rounding, the half-step bound, exactness where every step is exact, and an
+integer tie that e4m3 breaks.
+
 ``simulated_attention`` follows those steps in fp64 on quantised operands.
 The scheme is our reading (the pages define none), so it is a diagnostic: it
 separates the quantisation floor from kernel errors.  Its implementation of
@@ -90,14 +97,41 @@ def quantize_blocks(x: np.ndarray, block: int):
     return quantize_e4m3(x / rep[..., None]), sc
 
 
+INT8_MAX = 127.0
+
+
+def quantize_int8(x) -> np.ndarray:
+    """Symmetric int8: round x (fp64) to the nearest integer, ties to even, clipped to +-127."""
+    return np.clip(np.round(np.asarray(x, dtype=np.float64)), -INT8_MAX, INT8_MAX)
+
+
+def quantize_int8_blocks(x: np.ndarray, block: int):
+    """(int8 codes as fp64, scales) for per-block symmetric int8 quantisation of x [..., N, d]:
+    each block of `block` tokens of one (batch, head) gets scale amax / 127 (an all-zero
+    block gets 1), the reading of SageAttention's 8-bit Q and K."""
+    N = x.shape[-2]
+    nb = (N + block - 1) // block
+    sc = np.empty(x.shape[:-2] + (nb,), dtype=np.float64)
+    codes = np.empty_like(x, dtype=np.float64)
+    for i in range(nb):
+        blk = x[..., i * block:(i + 1) * block, :]
+        a = np.abs(blk).max(axis=(-2, -1))
+        sc[..., i] = np.where(a > 0, a / INT8_MAX, 1.0)
+        codes[..., i * block:(i + 1) * block, :] = quantize_int8(blk / sc[..., i, None, None])
+    return codes, sc
+
+
 def smooth_k(k: np.ndarray) -> np.ndarray:
     """K minus its per-(batch, head) channel mean over all tokens."""
     return k - k.mean(axis=-2, keepdims=True)
 
 
 def simulated_attention(q, k, v, scale=None, pos=None, axes=None, theta=10000.0,
-                        q_block=128, kv_block=64, smooth=True, rows=None):
-    """fp64 attention on e4m3-quantised operands (diagnostic of our FP8 reading)."""
+                        q_block=128, kv_block=64, smooth=True, rows=None, qk="e4m3"):
+    """fp64 attention on e4m3-quantised operands (diagnostic of our FP8 reading).
+
+    qk="int8" quantises Q and K to per-block symmetric int8 instead (SageAttention's
+    split: 8-bit integer Q.K^T, FP8 P.V); every other step is the same."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     if pos is not None:
         q = _rope.apply(q, pos, axes, theta)
@@ -106,8 +140,14 @@ def simulated_attention(q, k, v, scale=None, pos=None, axes=None, theta=10000.0,
         k = smooth_k(k)
     B, H, N, d = q.shape
     sigma = 1.0 / math.sqrt(d) if scale is None or scale <= 0 else float(scale)
-    q8, sq = quantize_blocks(q, q_block)
-    k8, sk = quantize_blocks(k, kv_block)
+    if qk == "e4m3":
+        q8, sq = quantize_blocks(q, q_block)
+        k8, sk = quantize_blocks(k, kv_block)
+    elif qk == "int8":
+        q8, sq = quantize_int8_blocks(q, q_block)
+        k8, sk = quantize_int8_blocks(k, kv_block)
+    else:
+        raise ValueError("qk must be 'e4m3' or 'int8'")
     v8, sv = quantize_blocks(v, kv_block)
     ridx = np.arange(N) if rows is None else np.asarray(rows)
     out = np.empty((B, H, len(ridx), d), dtype=np.float64)

@@ -1,4 +1,5 @@
 """Pins of the e4m3 quantiser and of the cache-gate oracle (no GPU)."""
+import dataclasses
 import json
 import math
 import os
@@ -101,6 +102,104 @@ def test_simulated_fp8_is_close_to_exact():
     s = fp8.simulated_attention(q, k, v)
     cos = (o * s).sum() / np.sqrt((o * o).sum() * (s * s).sum())
     assert cos > 0.995
+
+
+# --------------------------------------------------------------------------- int8
+# Symmetric per-block int8 for Q and K (SageAttention's 8-bit Q.K^T reading).
+def test_int8_codes_round_trip_ties_to_even_and_clip():
+    ints = np.arange(-127, 128, dtype=np.float64)
+    np.testing.assert_array_equal(fp8.quantize_int8(ints), ints)
+    mids = ints[:-1] + 0.5                                   # k + 1/2 for k = -127 .. 126
+    lo = np.floor(mids)
+    np.testing.assert_array_equal(fp8.quantize_int8(mids), np.where(lo % 2 == 0, lo, lo + 1))
+    np.testing.assert_array_equal(fp8.quantize_int8([127.5, 1e9, -127.5, -1e9]), [127, 127, -127, -127])
+
+
+def test_int8_matches_torch_round_and_clamp():
+    x = rng.uniform(-140.0, 140.0, 50000)
+    ref = torch.round(torch.from_numpy(x)).clamp(-127, 127).numpy()
+    np.testing.assert_array_equal(fp8.quantize_int8(x), ref)
+
+
+def test_int8_blocks_within_half_a_step():
+    """Blocks six orders of magnitude apart with planted amax: scales exactly amax / 127,
+    each block's amax on code +-127, every element within half a step (scale / 2), and
+    an all-zero block gets scale 1."""
+    x = rng.uniform(-1.0, 1.0, size=(1, 2, 300, 16))
+    mags = np.array([1e3, 1e-3, 1e3, 1e-3, 1.0])
+    amax = mags * 1.5
+    for b in range(5):
+        x[..., 64 * b:64 * (b + 1), :] *= mags[b]
+        x[..., 64 * b + 9, 5] = amax[b]
+    codes, sc = fp8.quantize_int8_blocks(x, 64)
+    np.testing.assert_array_equal(sc, np.broadcast_to(amax / 127.0, sc.shape))
+    rep = np.repeat(amax / 127.0, 64)[:300][None, None, :, None]
+    assert np.all(np.abs(codes * rep - x) <= 0.5 * rep * (1 + 1e-12))
+    for b in range(5):
+        assert np.abs(codes[..., 64 * b:64 * (b + 1), :]).max() == 127.0
+    assert fp8.quantize_int8_blocks(np.zeros((1, 1, 64, 4)), 64)[1][0, 0, 0] == 1.0
+
+
+def _int8_exact_inputs(N=192, seed=21):
+    """Inputs every step of the int8 reading represents exactly: integer Q, K with block
+    amax 127 (scale 1), e4m3 V with block amax 448 (scale 1, no V fold), and scores
+    k_j * ln 2 with k_j in [113, 127], so every P = 2^(k_j - 127) * 448 is an e4m3 value."""
+    g = np.random.default_rng(seed)
+    q = np.zeros((1, 1, N, 2))
+    q[..., 0] = 127.0                                          # every query row the same
+    k = np.zeros((1, 1, N, 2))
+    k[..., 0] = g.integers(113, 128, N)
+    k[..., 1] = g.integers(-127, 128, N)                       # meets q's zero channel
+    k[..., ::64, 0] = 127.0                                    # block amax 127
+    vals = _all_finite_values()
+    v = g.choice(vals[np.abs(vals) <= 448.0], size=(1, 1, N, 2))
+    v[..., ::64, 1] = 448.0                                    # block amax 448
+    return q, k, v, math.log(2.0) / 127.0
+
+
+def test_simulated_int8_is_exact_where_every_step_is():
+    q, k, v, sigma = _int8_exact_inputs()
+    exact = A.attention(q, k, v, scale=sigma)
+    sim = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False, qk="int8")
+    np.testing.assert_allclose(sim, exact, rtol=1e-13, atol=1e-13)
+    sim_e4m3 = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False)
+    assert np.abs(sim_e4m3 - exact).max() > 1e-3            # e4m3 Q.K^T is not exact here
+
+
+def test_simulated_int8_keeps_an_integer_tie():
+    """q = (127, 113) meets keys (127, 0) and (14, 127) with the same integer product
+    16129; every other key is 0 (score 40 lower, its P rounds to 0) and V picks e0 / e1.
+    The int8 reading, exact on these integers, gives (1/2, 1/2) on every row.  At scale
+    127/448, 113 and 14 fall off the e4m3 grid by different relative amounts, so
+    rounding Q, K or both to e4m3 breaks the tie."""
+    N = 64
+    q = np.zeros((1, 1, N, 2))
+    q[...] = (127.0, 113.0)
+    k = np.zeros((1, 1, N, 2))
+    k[0, 0, 0] = (127.0, 0.0)
+    k[0, 0, 1] = (14.0, 127.0)
+    v = np.zeros((1, 1, N, 2))
+    v[0, 0, 0] = (1.0, 0.0)
+    v[0, 0, 1] = (0.0, 1.0)
+    sigma = 40.0 / 16129.0
+    o = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False, qk="int8")
+    np.testing.assert_allclose(o, 0.5, rtol=0, atol=1e-13)
+    o8 = fp8.simulated_attention(q, k, v, scale=sigma, smooth=False)
+    assert np.abs(o8 - 0.5).max() > 1e-2
+
+
+def test_simulated_int8_meets_the_target_on_outliers():
+    """Diagnostic (not a pin): on the 1024-px outlier workload the int8 Q.K^T reading
+    reaches cosine >= 0.995 against exact attention, where e4m3 Q.K^T stays near 0.98."""
+    w = synth.WORKLOADS["flux1k"]
+    q, k, v = synth.qkv(dataclasses.replace(w, H=1))
+    pos = synth.positions(w.T, w.G).numpy()
+    rows = np.random.default_rng(4).integers(0, w.N, 128)
+    ex = A.attention(q, k, v, pos=pos, axes=w.axes, theta=w.theta, rows=rows)
+    cos = lambda a: float((a * ex).sum() / math.sqrt((a * a).sum() * (ex * ex).sum()))
+    i8 = fp8.simulated_attention(q, k, v, pos=pos, axes=w.axes, theta=w.theta, rows=rows, qk="int8")
+    e4 = fp8.simulated_attention(q, k, v, pos=pos, axes=w.axes, theta=w.theta, rows=rows)
+    assert cos(i8) >= 0.995 > cos(e4)
 
 
 # --------------------------------------------------------------------------- gate
@@ -318,3 +417,10 @@ def test_simulated_attention_pins_catch_planted_mistakes(name):
         except AssertionError:
             failed += 1
     assert failed >= 1, name
+
+
+@pytest.mark.parametrize("pin", _SIM_PINS, ids=lambda f: f.__name__[5:])
+def test_simulated_attention_int8_pins(pin):
+    """The closed forms and invariants hold for the int8 Q.K^T reading too."""
+    import functools
+    pin(functools.partial(fp8.simulated_attention, qk="int8"))

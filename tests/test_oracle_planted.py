@@ -141,6 +141,36 @@ def test_e4m3_pins_catch_planted_mistakes(name, monkeypatch):
     assert _count_failing(E4M3_PINS) >= 1, name
 
 
+INT8_PINS = [
+    T8.test_int8_codes_round_trip_ties_to_even_and_clip,
+    T8.test_int8_matches_torch_round_and_clamp,
+    T8.test_int8_blocks_within_half_a_step,
+    T8.test_simulated_int8_is_exact_where_every_step_is,
+    T8.test_simulated_int8_keeps_an_integer_tie,
+]
+
+INT8_MISTAKES = {
+    "ties_away_from_zero": [("np.clip(np.round(np.asarray(x, dtype=np.float64)), -INT8_MAX, INT8_MAX)",
+                             "np.clip(np.trunc(np.asarray(x, dtype=np.float64) + np.copysign(0.5, x)), "
+                             "-INT8_MAX, INT8_MAX)")],
+    "no_clip": [("np.clip(np.round(np.asarray(x, dtype=np.float64)), -INT8_MAX, INT8_MAX)",
+                 "np.round(np.asarray(x, dtype=np.float64))")],
+    "clip_at_128": [("INT8_MAX = 127.0", "INT8_MAX = 128.0")],
+    "amax_mapped_to_255": [("a / INT8_MAX, 1.0", "a / 255.0, 1.0")],
+    "zero_block_scale_zero": [("a / INT8_MAX, 1.0", "a / INT8_MAX, 0.0")],
+    "first_block_scale_for_all": [("quantize_int8(blk / sc[..., i, None, None])", "quantize_int8(blk / sc[..., 0, None, None])")],
+    "k_left_in_e4m3": [("        k8, sk = quantize_int8_blocks(k, kv_block)", "        k8, sk = quantize_blocks(k, kv_block)")],
+    "q_left_in_e4m3": [("        q8, sq = quantize_int8_blocks(q, q_block)", "        q8, sq = quantize_blocks(q, q_block)")],
+}
+
+
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")
+@pytest.mark.parametrize("name", sorted(INT8_MISTAKES))
+def test_int8_pins_catch_planted_mistakes(name, monkeypatch):
+    monkeypatch.setattr(T8, "fp8", _mutant(fp8, INT8_MISTAKES[name]))
+    assert _count_failing(INT8_PINS) >= 1, name
+
+
 GATE_PINS = [
     T8.test_golden_gate,
     T8.test_gate_brute_force_on_tiny_sweep,
@@ -182,4 +212,5 @@ def test_unmutated_copies_pass_every_pin(monkeypatch):
     assert _count_failing(ATTENTION_PINS) == 0
     assert _count_failing(ROPE_PINS) == 0
     assert _count_failing(E4M3_PINS) == 0
+    assert _count_failing(INT8_PINS) == 0
     assert _count_failing(GATE_PINS) == 0
