@@ -93,7 +93,7 @@ def _cos(a, b):
     return float((a * b).sum() / math.sqrt((a * a).sum() * (b * b).sum()))
 
 
-def _case(outliers, N=None):
+def _case(outliers):
     w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2, outliers=outliers)
     q, k, v = synth.qkv(w)
     pos = synth.positions(w.T, w.G).numpy()
