@@ -166,12 +166,38 @@ class ClockSampler:
 # ----------------------------------------------------------------------- CPU oracle legs
 def oracle_sample(q, k, v, pos, w, heads, rows):
     """Exact fp64 attention of the oracle on `heads` heads x `rows` query rows. Returns (flops, seconds)."""
+    import numpy as np
     from oracle import attention as A
     t0 = time.perf_counter()
     A.attention(q[:, :heads], k[:, :heads], v[:, :heads], pos=pos, axes=w.axes, theta=w.theta,
-                rows=None if rows >= w.N else __import__("numpy").arange(rows))
+                rows=None if rows >= w.N else np.arange(rows))
     dt = time.perf_counter() - t0
     return 4.0 * heads * rows * w.N * w.d, dt
+
+
+def cpu_baseline_leg(q, k, v, pos, w, seconds):
+    """The oracle on a bounded sample of the workload, on host tensors: whole heads
+    (all N query rows) on every BLAS thread until `seconds` of work, then one head x
+    512 rows on a single thread.  Returns the bench line's cpu_baseline object."""
+    f_tot, t_tot, heads = 0.0, 0.0, 0
+    while heads < w.H and (heads == 0 or t_tot < seconds):  # at least one head
+        f, dt = oracle_sample(q[:, heads:heads + 1], k[:, heads:heads + 1], v[:, heads:heads + 1], pos, w, 1, w.N)
+        f_tot += f
+        t_tot += dt
+        heads += 1
+    line = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"fp64 exact attention with RoPE on {heads} of {w.H} heads (all {w.N} query rows each), "
+                      f"{t_tot:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            rows = min(512, w.N)
+            f1, t1 = oracle_sample(q[:, :1], k[:, :1], v[:, :1], pos, w, 1, rows)
+        line["single_thread"] = {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                 "sample": f"1 head x {rows} query rows x {w.N} keys, {t1:.1f} s"}
+    except ImportError:
+        pass
+    return line
 
 
 def cpu_cores():
@@ -413,18 +439,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-        posn = pos.cpu().numpy()
-        f_tot, t_tot, heads = 0.0, 0.0, 0
-        while heads < H and t_tot < args.cpu_seconds:
-            f, dt = oracle_sample(qc[:, heads:heads + 1], kc[:, heads:heads + 1], vc[:, heads:heads + 1], posn, w,
-                                  1, N)
-            f_tot += f
-            t_tot += dt
-            heads += 1
-        cpu = {"value": f_tot / t_tot / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"fp64 exact attention with RoPE on {heads} of 24 heads (all 16896 query rows each), "
-                         f"{t_tot:.1f} s"}
+        cpu = cpu_baseline_leg(q.cpu(), k.cpu(), v.cpu(), pos.cpu().numpy(), w, args.cpu_seconds)
 
     if rank == 0:
         line = {

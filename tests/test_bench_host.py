@@ -54,3 +54,16 @@ def test_reference_arm_json_line():
 
 def test_reference_arm_other_ranks_print_nothing():
     assert _run_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_cpu_baseline_leg_reports_all_and_single_thread_figures():
+    from diffusion_transformer_denoising_dit_b200 import synth
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w)
+    pos = synth.positions(w.T, w.G).numpy()
+    line = bench.cpu_baseline_leg(q, k, v, pos, w, seconds=0.0)
+    assert line["kind"] == "oracle" and line["unit"] == "TFLOP/s" and line["value"] > 0 and line["cores"] >= 1
+    assert "1 of 2 heads" in line["sample"]          # always one head, more only while the budget lasts
+    assert "2 of 2 heads" in bench.cpu_baseline_leg(q, k, v, pos, w, seconds=60.0)["sample"]
+    st = line["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0 and "288 query rows" in st["sample"]
