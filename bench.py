@@ -5,9 +5,14 @@ One step = one pass of the hot path over the Flux-like 2048-px workload
 (B=1, H=24, N=512 text + 128x128 image = 16896 tokens, d=128):
 rotary embedding of K (one pass) and BF16 joint attention (which rotates Q as it
 loads each Q tile), and the First-Block-Cache gate on a 16896 x 3072 bf16
-hidden-state residual pair.  The FP8 variant (K rotation + smoothing + per-block
-e4m3 quantisation of K and V, then FP8 attention, which rotates and quantises Q
-as it loads it) is timed the same way and reported in the "fp8" object.
+hidden-state residual pair.  The two FP8 variants (a prologue that rotates Q and
+K, smooths K and quantises Q, K, V per block, then the 8-bit attention kernel:
+integer Q.K^T with int8 Q and K, or e4m3 Q.K^T) are timed the same way and
+reported in the "fp8" (integer Q.K^T) and "fp8_e4m3" objects.
+
+Inside each timed region every step's calls are bracketed by CUDA events on
+the launching stream, so the per-call times the roofline uses come from the
+same steps (and the same clocks) as the headline value.
 
 value = attention FLOPs (4*B*H*N^2*d per call) x calls / device time, in
 TFLOP/s, summed over ranks (each rank runs its own independent problem: weak
@@ -37,17 +42,16 @@ WORKLOAD = "flux2k"
 HIDDEN = 3072
 THRESHOLD = 0.12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Dense e4m3 GEMM (cuBLASLt via torch._scaled_mm, 8192^3) measured on this machine with
-# `python bench.py --measure-fp8-peak` (profiles/fp8_gemm_peak.md); reported beside
-# the nominal-ratio FP8 peak, which stays the roofline denominator.
-FP8_GEMM_MEASURED = {"burst": 3132.4, "sustained": 2594.0}
+# Sustained dense e4m3 GEMM (cuBLASLt via torch._scaled_mm, 8192^3, a 4 s loop under
+# the power cap), recorded from `python bench.py --measure-fp8-peak` on this pool;
+# the burst figure is measured live in every run.
+FP8_GEMM_SUSTAINED_RECORDED = 2594.0
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel, keyed
-# by the hash of the kernel source it was taken on (code only, comments ignored);
-# a changed kernel reports null.
+# by the hash of the kernel source it was taken on (code only, comments ignored).
+# These are capture results, not measurements of this run; a kernel whose source
+# changed since its capture reports null.
 NCU_TRAFFIC = {
-    # profiles/attn_bf16_flux2k.md: 323.0 MB read + 87.0 MB written per launch
-    ("attn_bf16", "b620164e5e13027b"): 409_936_384,
 }
 
 
@@ -266,81 +270,89 @@ def run_ours(args, rank, world, local_rank):
     o = torch.empty_like(q)
     ws = dit.attention_workspace(B, H, N, d, "bf16", rope=True, device=dev)
     gate = dit.FBCacheGate(THRESHOLD, r_cur.numel(), device=dev)
-    have_fp8 = True
-    try:
-        ws8 = dit.attention_workspace(B, H, N, d, "fp8", device=dev)
-        dit.attention(q, k, v, cos, sin, precision="fp8", out=o, workspace=ws8)
-    except dit.DitError:
-        have_fp8 = False
+    fp8_kinds = {}
+    for prec in ("fp8_i8qk", "fp8"):
+        try:
+            ws8 = dit.attention_workspace(B, H, N, d, prec, device=dev)
+            dit.attention(q, k, v, cos, sin, precision=prec, out=o, workspace=ws8)
+            fp8_kinds[prec] = ws8
+        except dit.DitError:
+            pass
 
-    def step_bf16():
-        dit.attention(q, k, v, cos, sin, out=o, workspace=ws)
-        gate(r_cur, r_prev)
-
-    def step_fp8():
-        dit.attention(q, k, v, cos, sin, precision="fp8", out=o, workspace=ws8)
-        gate(r_cur, r_prev)
-
-    def timed(fn, steps, warmup):
+    def timed(calls, steps, warmup):
+        """Runs `steps` steps, each the sequence of (name, fn) calls, after `warmup`
+        untimed ones.  Returns the whole region's device time (ms) and, per call
+        name, the median of its per-step device times (ms), from CUDA events on the
+        launching stream recorded around every call of every timed step."""
         for _ in range(warmup):
-            fn()
+            for _, fn in calls:
+                fn()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(steps):
-            fn()
+        for t in range(steps):
+            ev[t][0].record(stream)
+            for c, (_, fn) in enumerate(calls):
+                fn()
+                ev[t][c + 1].record(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        return e0.elapsed_time(e1)
+        med = lambda xs: sorted(xs)[len(xs) // 2]
+        per = {name: med([ev[t][c].elapsed_time(ev[t][c + 1]) for t in range(steps)])
+               for c, (name, _) in enumerate(calls)}
+        return e0.elapsed_time(e1), per
 
     def max_over_ranks(x):
         return gather_floats(x, world, dev)
 
-    # ---- main timed region: BF16 step (rotary + attention + gate)
+    def mcycles(ms, clk):
+        return None if not clk.get("sm_mhz") else ms * clk["sm_mhz"] / 1e3
+
+    bf16_calls = [("attention", lambda: dit.attention(q, k, v, cos, sin, out=o, workspace=ws)),
+                  ("gate", lambda: gate(r_cur, r_prev))]
+
+    # ---- main timed region: BF16 step (rotary K pass + attention + gate)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-        ms = timed(step_bf16, args.steps, args.warmup)
+        ms, per = timed(bf16_calls, args.steps, args.warmup)
     clocks = clk.summary()
     all_ms = max_over_ranks(ms)
     value, ms_per_step = aggregate(all_ms, [flops * args.steps] * world, args.steps)
     assert dit.read_error() == 0
 
-    # ---- dominant kernel: the attention launch with RoPE fused into its Q load.  The
-    # call is the K rotation pass followed by that launch; the K pass (the same kernel
-    # on the same tensor) is timed alone and subtracted.
-    # The three are timed in alternation over several rounds (medians), so that clock
-    # drift under the power cap does not bias the difference.
-    ka = max(5, args.steps)
-    kr2 = torch.empty_like(k)
-    t_call, t_rope, t_plain = [], [], []
-    for _ in range(5):
-        t_call.append(timed(lambda: dit.attention(q, k, v, cos, sin, out=o, workspace=ws), ka, 2) / ka)
-        t_rope.append(timed(lambda: dit.rope_apply(k, cos, sin, out=kr2), ka, 2) / ka)
-        # for reference: one launch on pre-rotated Q/K without tables (no in-kernel rotation)
-        t_plain.append(timed(lambda: dit.attention(q, kr2, v, out=o), ka, 2) / ka)
-    med = lambda xs: sorted(xs)[len(xs) // 2]
-    ms_call, ms_rope, ms_plain = med(t_call), med(t_rope), med(t_plain)
-    ms_attn = ms_call - ms_rope
-    achieved = flops / (ms_attn / 1e3) / 1e12
+    # ---- dominant kernel: the attention call of those same steps (the K rotation
+    # pass, about 2 % of it, then the attention kernel, which rotates Q as it loads
+    # it), so its per-launch time never exceeds the step time it is part of.
+    ms_call = per["attention"]
+    achieved = flops / (ms_call / 1e3) / 1e12
     bf16_peak = peaks["bf16_tflops"]
     h_attn = _src_hash("attn_kernel.cuh", "dit_device.cuh", "attn_bf16.cu")
     tr = NCU_TRAFFIC.get(("attn_bf16", h_attn))
-    roofline = {"bound": "tensor", "kernel": "attn_kernel<bf16, d=128>", "achieved": achieved, "peak": bf16_peak,
+    roofline = {"bound": "tensor", "kernel": "attn_kernel<bf16, d=128> (+ the K rotation pass of the same call)",
+                "achieved": achieved, "peak": bf16_peak,
                 "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": tr,
+                "traffic_source": (f"ncu capture of this kernel source (hash {h_attn})" if tr is not None
+                                   else f"no capture of this kernel source (hash {h_attn})"),
                 "peak_source": f"{peak_kind} bf16 burst (cuBLAS 8192^3)",
                 "frac_of_nominal_2250": achieved / 2250.0,
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", bf16_peak),
-                "ms_per_launch": ms_attn,
-                "ms_per_launch_how": "median over 5 alternating rounds: attention call with RoPE minus the K "
-                                     "rotation pass timed alone",
-                "ms_per_launch_prerotated_no_tables": ms_plain}
+                "ms_per_launch": ms_call,
+                "ms_per_launch_how": "median over the timed steps of CUDA events around the attention call "
+                                     "(K rotation pass + attention kernel) inside the headline region",
+                "sm_mcycles_per_launch": mcycles(ms_call, clocks)}
 
-    # ---- side kernels alone: rotary pre-pass of K (timed above) and the gate (HBM-bound)
+    # ---- side kernels alone (HBM-bound): the K rotation pass and the gate
+    kr2 = torch.empty_like(k)
+    ka = max(5, args.steps)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk_side:
+        _, per_side = timed([("rope", lambda: dit.rope_apply(k, cos, sin, out=kr2)),
+                             ("gate", lambda: gate(r_cur, r_prev))], ka, 3)
+    ms_rope, ms_gate = per_side["rope"], per_side["gate"]
     rope_bytes = 2 * k.numel() * 2 + 2 * cos.numel() * 4
-    ms_gate = timed(lambda: gate(r_cur, r_prev), ka, 3) / ka
     gate_bytes = 2 * r_cur.numel() * 2
     hbm = peaks["hbm_gbs"]
     side = {
@@ -348,24 +360,45 @@ def run_ours(args, rank, world, local_rank):
                        "ms": ms_rope, "bytes": rope_bytes},
         "fbcache_gate": {"GB/s": gate_bytes / (ms_gate / 1e3) / 1e9,
                          "frac": gate_bytes / (ms_gate / 1e3) / 1e9 / hbm, "ms": ms_gate, "bytes": gate_bytes},
+        "clocks": clk_side.summary(),
+        "how": "medians of per-call CUDA events over a region of alternating rope_apply(K) and gate calls",
     }
+    # the attention kernel alone, estimated: the call minus the K rotation pass timed above
+    roofline["kernel_only_estimate"] = {
+        "ms": ms_call - ms_rope, "TFLOP/s": flops / ((ms_call - ms_rope) / 1e3) / 1e12,
+        "frac": flops / ((ms_call - ms_rope) / 1e3) / 1e12 / bf16_peak,
+        "how": "attention call of the headline steps minus the median K rotation pass of the side-kernel region"}
 
-    # ---- FP8 step
-    fp8 = None
-    if have_fp8:
-        ms8 = timed(step_fp8, args.steps, args.warmup)
+    # ---- FP8 steps (prologue + 8-bit attention + gate), each in a region of its own
+    fp8_gemm = measure_fp8_gemm_burst(dev)
+    fp8_objs = {}
+    for prec, ws8 in fp8_kinds.items():
+        calls = [("attention", lambda ws8=ws8, prec=prec: dit.attention(q, k, v, cos, sin, precision=prec, out=o,
+                                                                        workspace=ws8)),
+                 ("gate", lambda: gate(r_cur, r_prev))]
+        with ClockSampler(dev.index if dev.index is not None else 0) as clk8:
+            ms8, per8 = timed(calls, args.steps, args.warmup)
+        c8 = clk8.summary()
         all8 = max_over_ranks(ms8)
         v8, mps8 = aggregate(all8, [flops * args.steps] * world, args.steps)
         fp8_peak = 2.0 * bf16_peak
-        fp8_sus = 2.0 * peaks.get("bf16_tflops_sustained", bf16_peak)
-        fp8 = {"value": v8 / 1e12, "unit": "TFLOP/s", "ms_per_step": mps8,
-               "peak": fp8_peak, "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
-               "frac_of_step": v8 / 1e12 / fp8_peak,
-               "peak_sustained": fp8_sus, "frac_of_step_vs_sustained": v8 / 1e12 / fp8_sus,
-               "measured_fp8_gemm": FP8_GEMM_MEASURED,
-               "frac_of_step_vs_measured_fp8_gemm": v8 / 1e12 / FP8_GEMM_MEASURED["burst"],
-               "frac_of_step_vs_measured_fp8_gemm_sustained": v8 / 1e12 / FP8_GEMM_MEASURED["sustained"]}
+        call8 = per8["attention"]
+        fp8_objs[prec] = {
+            "value": v8 / 1e12, "unit": "TFLOP/s", "ms_per_step": mps8,
+            "qk": "int8 (kind::i8, s32 accumulation)" if prec == "fp8_i8qk" else "e4m3 (kind::f8f6f4)",
+            "pv": "e4m3", "ms_per_call": call8,
+            "call_TFLOP/s": flops / (call8 / 1e3) / 1e12,
+            "measured_fp8_gemm_burst": fp8_gemm,
+            "frac_of_step_vs_measured_fp8_gemm": v8 / 1e12 / fp8_gemm if fp8_gemm else None,
+            "frac_of_call_vs_measured_fp8_gemm": flops / (call8 / 1e3) / 1e12 / fp8_gemm if fp8_gemm else None,
+            "fp8_gemm_sustained_recorded": FP8_GEMM_SUSTAINED_RECORDED,
+            "frac_of_step_vs_fp8_gemm_sustained": v8 / 1e12 / FP8_GEMM_SUSTAINED_RECORDED,
+            "peak_nominal_ratio": fp8_peak, "frac_of_step_vs_2x_bf16": v8 / 1e12 / fp8_peak,
+            "clocks": c8, "sm_mcycles_per_step": mcycles(mps8, c8),
+            "step": f"{prec} call (prologue + attention) + fbcache_gate"}
         assert dit.read_error() == 0
+    fp8 = fp8_objs.get("fp8_i8qk")
+    fp8_e4m3 = fp8_objs.get("fp8")
 
     # ---- e2e through the public API from pinned host buffers.  Every step copies its
     # inputs (Q, K, V and the two gate residuals) host -> device and reads its output
@@ -456,7 +489,9 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": f"independent problem per rank x{world}"},
             "roofline": roofline,
             "fp8": fp8,
+            "fp8_e4m3": fp8_e4m3,
             "side_kernels": side,
+            "sm_mcycles_per_step": mcycles(ms_per_step, clocks),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": max(all_e2e) / ke,
@@ -533,13 +568,14 @@ def run_trace(args):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1), calls, skipped, [a.elapsed_time(b) for a, b in per_step]
 
-    def run_device():
-        """The same trace with the decision left on the device: every step enqueues
-        block 0, the gate and the 56 remaining calls as skippable launches driven by
-        the gate's flag, with no host read inside the loop (a skipped step costs
-        56 pairs of launches that return at once).  The per-step flags are copied
-        to a device array and read once at the end."""
-        never = torch.zeros(1, dtype=torch.int32, device=dev)
+    def run_device(policy="consecutive"):
+        """The same trace with the decision and the reference residual left on the
+        device (FBCacheGate.step): every step enqueues block 0, the gate and the 56
+        remaining calls as skippable launches driven by the gate's flag, with no
+        host read inside the loop (a skipped step costs 56 pairs of launches that
+        return at once).  The per-step flags are copied to a device array and read
+        once at the end."""
+        g = dit.FBCacheGate(thr, res[0].numel(), device=dev, policy=policy)
         flags = torch.zeros(steps, dtype=torch.int32, device=dev)
         torch.cuda.synchronize()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -548,7 +584,7 @@ def run_trace(args):
         for t in range(steps):
             attn(calls)
             calls += 1
-            flag = gate(res[t], res[t - 1]) if t > 0 else never
+            flag = g.step(res[t])
             flags[t:t + 1].copy_(flag)
             for _ in range(blocks - 1):
                 q, k, v = sets[calls % 4]
@@ -565,6 +601,7 @@ def run_trace(args):
     gated_ms, gated_calls, skipped, gated_steps = run(True)
     dev_ms, dev_skipped = run_device()
     last_ms, last_calls, last_skipped, _ = run(True, policy="last_computed")
+    dev_last_ms, dev_last_skipped = run_device("last_computed")
     assert dit.read_error() == 0
     line = {
         "metric": "28-step 2048px denoising attention trace with First-Block-Cache (threshold %.2f)" % thr,
@@ -577,14 +614,47 @@ def run_trace(args):
                     "rel_per_step": rel_seen},
         "speedup": base_ms / gated_ms,
         "fbcache_device_decision": {"ms": dev_ms, "skipped_steps": dev_skipped,
-                                    "how": "dit.attention(..., skip=gate flag) for blocks 1..56; no host "
-                                           "read inside the 28-step loop"},
+                                    "how": "FBCacheGate.step + dit.attention(..., skip=gate flag) for blocks "
+                                           "1..56; no host read inside the 28-step loop"},
         "speedup_device_decision": base_ms / dev_ms,
         "fbcache_last_computed": {"ms": last_ms, "attention_calls": last_calls, "skipped_steps": last_skipped,
                                   "how": "each step compared with the last step whose remaining blocks ran"},
         "speedup_last_computed": base_ms / last_ms,
+        "fbcache_last_computed_device_decision": {"ms": dev_last_ms, "skipped_steps": dev_last_skipped,
+                                                  "how": "FBCacheGate(policy='last_computed').step: the reference "
+                                                         "residual refreshed on the device only after computed steps"},
+        "speedup_last_computed_device_decision": base_ms / dev_last_ms,
     }
     print(json.dumps(line), flush=True)
+
+
+def measure_fp8_gemm_burst(dev):
+    """Dense e4m3 GEMM burst throughput (TFLOP/s) of the library (cuBLASLt through
+    torch._scaled_mm), 8192^3 with bf16 output, best of 10: the denominator of the
+    FP8 fractions, measured in the run that reports them."""
+    import torch
+    try:
+        n = 8192
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            mm()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mm()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
 
 
 def run_fp8_peak():

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     attention_workspace,
     fbcache_gate,
     fbcache_gate_finalize,
+    fbcache_gate_ref_update,
     fbcache_gate_sums,
     fp8_workspace_views,
     lib,

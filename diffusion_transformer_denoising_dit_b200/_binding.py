@@ -19,8 +19,9 @@ STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "D
           4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT"}
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
-           "dit_attn_fp8", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
-           "dit_selftest_wait_timeout", "dit_attn_bf16_skippable", "fbcache_gate_sums", "fbcache_gate_finalize"]
+           "dit_attn_fp8", "dit_attn_fp8_i8qk", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
+           "dit_selftest_wait_timeout", "dit_attn_bf16_skippable", "fbcache_gate_sums", "fbcache_gate_finalize",
+           "fbcache_gate_ref_update"]
 
 
 class DitError(RuntimeError):
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_fp8.restype = _i
         L.dit_attn_fp8.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64x3, _i64x3, _i64x3, _i64x3,
                                    _vp, _vp, ctypes.c_float, _i, _i, _i, _vp, _sz, _vp]
+        L.dit_attn_fp8_i8qk.restype = _i
+        L.dit_attn_fp8_i8qk.argtypes = L.dit_attn_fp8.argtypes
         L.fbcache_gate_workspace_bytes.restype = _sz
         L.fbcache_gate_workspace_bytes.argtypes = [ctypes.c_int64]
         L.fbcache_gate.restype = _i
@@ -76,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.fbcache_gate_sums.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, _sz, _vp]
         L.fbcache_gate_finalize.restype = _i
         L.fbcache_gate_finalize.argtypes = [_vp, ctypes.c_float, _vp, _vp, _vp]
+        L.fbcache_gate_ref_update.restype = _i
+        L.fbcache_gate_ref_update.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp]
         L.fbcache_gate_noalloc.restype = _i
         L.fbcache_gate_noalloc.argtypes = [_vp, _vp, ctypes.c_int64, ctypes.c_float, _vp, _vp, _vp]
         _lib = L
@@ -188,6 +193,9 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
               skip=None):
     """Joint attention O [B,H,N,d] bf16 from bf16 q, k, v (+ optional rotary tables).
 
+    precision: "bf16"; "fp8" (e4m3 Q, K, V and P); "fp8_i8qk" (symmetric int8 Q
+    and K with an integer Q.K^T, e4m3 V and P).  Both 8-bit forms share one
+    workspace layout.
     skip (BF16 only): a device int32 flag, e.g. FBCacheGate's output; when it is
     non-zero at the time the kernels run, the call does nothing and ``out`` keeps
     its previous contents."""
@@ -209,10 +217,10 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
     L = lib()
     if precision == "bf16":
         need = L.dit_attn_bf16_workspace_bytes(B, H, N, d, int(cos is not None))
-    elif precision == "fp8":
+    elif precision in ("fp8", "fp8_i8qk"):
         need = L.dit_attn_fp8_workspace_bytes(B, H, N, d, q_block, kv_block)
     else:
-        raise ValueError("precision must be 'bf16' or 'fp8'")
+        raise ValueError("precision must be 'bf16', 'fp8' or 'fp8_i8qk'")
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
     wp = _ptr(workspace) if need else None
@@ -223,14 +231,18 @@ def attention(q, k, v, cos=None, sin=None, precision: str = "bf16", scale: float
         _check("dit_attn_bf16_skippable", L.dit_attn_bf16_skippable(*args, wp, wb, skip.data_ptr(), _stream(q)))
     elif precision == "bf16":
         _check("dit_attn_bf16", L.dit_attn_bf16(*args, wp, wb, _stream(q)))
-    else:
+    elif precision == "fp8":
         _check("dit_attn_fp8", L.dit_attn_fp8(*args, q_block, kv_block, int(smooth_k), wp, wb, _stream(q)))
+    else:
+        _check("dit_attn_fp8_i8qk", L.dit_attn_fp8_i8qk(*args, q_block, kv_block, int(smooth_k), wp, wb, _stream(q)))
     return out
 
 
 def attention_workspace(B, H, N, d, precision="bf16", rope=True, q_block=128, kv_block=64, device="cuda"):
     """Pre-allocated workspace for repeated attention calls of one shape."""
     L = lib()
+    if precision not in ("bf16", "fp8", "fp8_i8qk"):
+        raise ValueError("precision must be 'bf16', 'fp8' or 'fp8_i8qk'")
     need = (L.dit_attn_bf16_workspace_bytes(B, H, N, d, int(rope)) if precision == "bf16"
             else L.dit_attn_fp8_workspace_bytes(B, H, N, d, q_block, kv_block))
     return torch.empty(max(need, 1), device=device, dtype=torch.uint8)
@@ -242,8 +254,9 @@ def _a256(x: int) -> int:
 
 def fp8_workspace_views(ws: torch.Tensor, B: int, H: int, N: int, d: int = 128, q_block: int = 128,
                         kv_block: int = 64):
-    """Views into a dit_attn_fp8 workspace (the layout written by the FP8 prologue):
-    q8, k8, v8 (uint8 e4m3 codes [B,H,N,d]), q_scale, k_scale, v_scale, k_mean, v_scale_max."""
+    """Views into a dit_attn_fp8 / dit_attn_fp8_i8qk workspace (the layout written by the
+    prologue): q8, k8, v8 (uint8 codes [B,H,N,d]: e4m3, or int8 two's complement for q8 and
+    k8 of the integer Q.K^T form), q_scale, k_scale, v_scale, k_mean, v_scale_max."""
     bh = B * H
     el = bh * N * d
     nq, nk = -(-N // q_block), -(-N // kv_block)
@@ -333,20 +346,75 @@ def fbcache_gate_finalize(sums, threshold: float, rel_out=None, skip_out=None):
     return rel_out, skip_out
 
 
+def fbcache_gate_ref_update(r_cur, r_ref, skip=None):
+    """r_ref <- r_cur on the device, unless the device int32 flag `skip` is set when
+    the copy runs (then r_ref keeps the last computed step's residual)."""
+    _need_cuda(r_cur, r_ref, skip)
+    if r_cur.dtype != torch.bfloat16 or r_ref.dtype != torch.bfloat16 or r_cur.numel() != r_ref.numel():
+        raise ValueError("r_cur, r_ref must be bf16 tensors of equal size")
+    if not r_cur.is_contiguous() or not r_ref.is_contiguous():
+        raise ValueError("r_cur, r_ref must be contiguous")
+    if skip is not None and (skip.dtype != torch.int32 or skip.numel() < 1):
+        raise ValueError("skip must be a CUDA int32 flag")
+    _check("fbcache_gate_ref_update", lib().fbcache_gate_ref_update(r_cur.data_ptr(), r_ref.data_ptr(), r_cur.numel(),
+                                                                    _ptr(skip), _stream(r_cur)))
+    return r_ref
+
+
 class FBCacheGate:
     """First-Block-Cache decision with its buffers allocated once.
 
-    gate(r_cur, r_prev) enqueues the kernels and returns the device int32
-    skip flag; ``.rel`` holds the relative L1 change.  Reading the flag on the
-    host (``bool(flag.item())``) is the one device-to-host crossing per step.
+    gate(r_cur, r_prev) enqueues the kernels for an explicit pair and returns the
+    device int32 skip flag; ``.rel`` holds the relative L1 change.
+
+    gate.step(r_cur) is the per-denoising-step form, with the reference held on
+    the device: policy "consecutive" compares every step with the step before it,
+    "last_computed" with the last step whose remaining blocks ran (so small
+    changes add up across skipped steps); the first ``warmup`` steps (at least
+    one: step 0 has nothing to compare with) are always computed.  The returned
+    flag drives the skippable attention call directly; nothing is read on the
+    host.  Reading it there (``bool(flag.item())``) is the one device-to-host
+    crossing per step when the caller branches on the host instead.
     """
 
-    def __init__(self, threshold: float, numel: int, device="cuda"):
+    POLICIES = ("consecutive", "last_computed")
+
+    def __init__(self, threshold: float, numel: int, device="cuda", policy: str = "consecutive", warmup: int = 1):
+        if policy not in self.POLICIES:
+            raise ValueError(f"policy must be one of {self.POLICIES}")
         self.threshold = float(threshold)
+        self.policy = policy
+        self.warmup = max(1, int(warmup))
+        self.numel = int(numel)
         self.rel = torch.empty(1, device=device, dtype=torch.float32)
         self.skip = torch.empty(1, device=device, dtype=torch.int32)
+        self.never = torch.zeros(1, device=device, dtype=torch.int32)
         self.workspace = torch.empty(lib().fbcache_gate_workspace_bytes(numel), device=device, dtype=torch.uint8)
+        self.ref = None
+        self.t = 0
 
     def __call__(self, r_cur, r_prev):
         fbcache_gate(r_cur, r_prev, self.threshold, self.rel, self.skip, self.workspace)
         return self.skip
+
+    def reset(self):
+        """Start a new denoising trajectory (the next step is step 0)."""
+        self.t = 0
+
+    def step(self, r_cur):
+        """Decision for this step's first-block residual r_cur: the device int32 flag
+        (1 = skip the remaining blocks).  Updates the device-side reference."""
+        if r_cur.numel() != self.numel:
+            raise ValueError(f"r_cur must have {self.numel} elements")
+        if self.ref is None:
+            self.ref = torch.empty(self.numel, device=r_cur.device, dtype=torch.bfloat16)
+        flat = r_cur.reshape(-1)
+        if self.t < self.warmup:
+            flag = self.never
+            fbcache_gate_ref_update(flat, self.ref)
+        else:
+            fbcache_gate(flat, self.ref, self.threshold, self.rel, self.skip, self.workspace)
+            flag = self.skip
+            fbcache_gate_ref_update(flat, self.ref, None if self.policy == "consecutive" else flag)
+        self.t += 1
+        return flag

@@ -6,6 +6,8 @@
 // Sources: "FLUX 3 Image Klein / TensorRT-LLM VisualGen" (cuDNN FP8 attention
 // against VANILLA BF16 on B200) and "vflash / Optimization ledger", table
 // "Accepted or exposed" (SageAttention2, quantised attention).
+// With Q and K in symmetric int8 (the prologue's qk_int8 mode) S = Q8 K8^T is
+// a kind::i8 MMA with s32 accumulation instead, scaled the same way.
 // The kernel itself is the shared template in attn_kernel.cuh.
 #include "attn_kernel.cuh"
 
@@ -19,6 +21,7 @@ cudaError_t launch_attn_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const 
   sc.v_scale = p.v_scale;
   sc.v_scale_max = p.v_scale_max;
   sc.H = p.H;
+  if (p.qk_int8) return launch_attn<true, 128, true>(tq, tk, tv, out, sc, p.B, p.H, stream);
   return launch_attn<true, 128>(tq, tk, tv, out, sc, p.B, p.H, stream);
 }
 

@@ -69,8 +69,8 @@ struct AttnCfg {
   static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
   static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
   static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2;
-  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 16;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 32;
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
   static constexpr uint32_t kTmemCols = 512;
@@ -90,6 +90,20 @@ struct AttnCfg {
   // whose MMAs are half as long, does better letting them exponentiate at the
   // same time (1.4 % fewer cycles).
   static constexpr bool kPingPong = !FP8;
+  // Exponentials computed on the FMA pipe (ex2_poly_pair) instead of the MUFU
+  // unit: bit e set = key pair e of each 32-key group (BF16, e < 16) or key quad e
+  // of each 32-key group, over two groups (FP8, bits 0-15).
+#ifdef DIT_POLY_MASK_BF16
+  static constexpr uint32_t kPolyMaskBf16 = DIT_POLY_MASK_BF16;
+#else
+  static constexpr uint32_t kPolyMaskBf16 = 0u;
+#endif
+#ifdef DIT_POLY_MASK_FP8
+  static constexpr uint32_t kPolyMaskFp8 = DIT_POLY_MASK_FP8;
+#else
+  static constexpr uint32_t kPolyMaskFp8 = 0u;
+#endif
+  static constexpr uint32_t kPolyMask = FP8 ? kPolyMaskFp8 : kPolyMaskBf16;
   static constexpr float kRescaleLog2 = static_cast<float>(kTau);
   static constexpr float kTwoTau = static_cast<float>(1ull << kTau);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -111,6 +125,17 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Integer score -> float without a conversion instruction: for |s| < 2^22 the
+// bits (s & 0x7FFFFF) ^ 0x4B400000 are the float 1.5 * 2^23 + s, exactly (one
+// lop3).  The softmax works on these biased values and folds the bias into
+// its scale-and-subtract constant.
+constexpr float kI8Bias = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint32_t s32_biased_f32(uint32_t s) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, 0x007FFFFF, 0x4B400000, 0x6A;" : "=r"(r) : "r"(s));
+  return r;
 }
 
 __device__ __forceinline__ float lg2(float x) {
@@ -136,7 +161,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 // serialised sixteen round trips (about 16k cycles per CTA, measured).
 // Out of line, so that its registers stay out of the softmax branch's allocation.
 template <int D, typename Wait>
-__device__ __noinline__ void rotate_q_tile(uint8_t* q_tile, const float* rope_cos, const float* rope_sin, int qrow0,
+__device__ __noinline__ bool rotate_q_tile(uint8_t* q_tile, const float* rope_cos, const float* rope_sin, int qrow0,
                                            int N, Wait wait_tile) {
   constexpr int kSubBytes = 128 * 128;  // one 128-row, 128-byte column block
   constexpr int CPR = D / 8;            // 16-byte chunks per row
@@ -158,7 +183,7 @@ __device__ __noinline__ void rotate_q_tile(uint8_t* q_tile, const float* rope_co
     }
   }
   const bool q_ok = wait_tile();
-  if (!rope || !q_ok) return;
+  if (!rope || !q_ok) return q_ok;
 #pragma unroll
   for (int k = 0; k < NP; ++k) {
     // row r's chunk c sits at column block c / 8, 16-byte slot (c % 8) ^ (r % 8) (128-byte swizzle)
@@ -181,12 +206,16 @@ __device__ __noinline__ void rotate_q_tile(uint8_t* q_tile, const float* rope_co
     o4.w = pack_bf16x2(y[6], y[7]);
     *p = o4;
   }
+  return true;
 }
 
-template <bool FP8, int D>
+// I8QK (FP8 only): Q and K are symmetric int8 and S = Q K^T is a kind::i8 MMA
+// with s32 accumulation (exact: |S| <= 127^2 * 128 < 2^22); P.V stays e4m3.
+template <bool FP8, int D, bool I8QK = false>
 __global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnOut out, const AttnScales sc) {
+  static_assert(FP8 || !I8QK, "the integer Q.K^T belongs to the FP8 variant");
   using C = AttnCfg<FP8, D>;
   constexpr int NK = C::NK, NV = C::NV, BM = C::BM, BN = C::BN;
   // device-side skip (the cache gate's flag): the whole CTA leaves before any
@@ -203,13 +232,30 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_full = k_empty + NK;
   uint64_t* v_empty = v_full + NV;
   uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and every earlier MMA)
-  uint64_t* pv_done = s_full + 2;    // [2] PV_i(j) computed (read by the epilogue)
+  uint64_t* pv_done = s_full + 2;    // [2] the last PV_i computed (read by the epilogue)
   uint64_t* q_ready = pv_done + 2;   // [2] BF16: Q_i rotated in shared memory (128 arrivals)
+  uint64_t* mma_drain = q_ready + 2; // failure path: every MMA the MMA thread issued has completed
   // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
   //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
   //                 kBarPHalf + i   BF16: softmax i stored keys 0..63 of P (128 arrive, MMA warp syncs)
   constexpr uint32_t kBarPReady = 1, kBarTurn = 3, kBarPHalf = 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
+  // Raised by the first role whose bounded wait gives up; every other bounded
+  // wait then gives up too.  A role that gives up still performs the rest of its
+  // named-barrier schedule (arrivals and syncs, without the work between them),
+  // so a partner blocked on a named barrier is always released: named barriers
+  // cannot time out, and their schedule is balanced.
+  const uint32_t abort_flag = smem_u32(tmem_slot + 1);
+  // Progress counters that pace the failure path (written on every path, read only
+  // on the failure path): mma_done[i] = PReady_i generations the MMA warp has
+  // passed.  A warpgroup on the failure path makes an arrival only once its
+  // partner has passed the previous generation of that barrier, as the data
+  // dependencies ensure on the normal path, so that no arrival lands a
+  // generation early (a named barrier would merge it into the current generation
+  // and strand the partner).  The MMA warp's progress also bounds the ping-pong
+  // partner's: it passes PReady_1(t-1) only after warpgroup 1 passed Turn_1(t-1),
+  // and PReady_0(t) only after warpgroup 0 passed Turn_0(t-1).
+  const uint32_t mma_done = smem_u32(tmem_slot + 2);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -219,6 +265,10 @@ __global__ void __launch_bounds__(384, 1)
   int* err = out.err;
 
   if (threadIdx.x == 0) {
+    flag_store(abort_flag, 0);
+    flag_store(mma_done, 0);
+    flag_store(mma_done + 4, 0);
+    mbar_init(mma_drain, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(s_full + i, 1);
@@ -260,25 +310,41 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sQ + i * C::kTileBytes + c * C::kSubBytes, &tmQ, q_full + i, c * C::kBoxInner,
                       (2 * qt + i) * BM, h, b);
       }
+      int nk_issued = 0, nv_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int sk = j % NK, sv = j % NV;
-        if (j >= NK && !mbar_wait(k_empty + sk, ((j / NK) & 1) ^ 1, err, kErrTimeout)) break;
+        if (j >= NK && !mbar_wait(k_empty + sk, ((j / NK) & 1) ^ 1, err, kErrTimeout, abort_flag)) break;
         mbar_arrive_expect_tx(k_full + sk, C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
           tma_load_4d(sK + sk * C::kTileBytes + c * C::kSubBytes, &tmK, k_full + sk, c * C::kBoxInner, j * BN, h, b);
-        if (j >= NV && !mbar_wait(v_empty + sv, ((j / NV) & 1) ^ 1, err, kErrTimeout)) break;
+        ++nk_issued;
+        if (j >= NV && !mbar_wait(v_empty + sv, ((j / NV) & 1) ^ 1, err, kErrTimeout, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + sv, C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
           tma_load_4d(sV + sv * C::kTileBytes + c * C::kSubBytes, &tmV, v_full + sv, c * C::kBoxInner, j * BN, h, b);
+        ++nv_issued;
+      }
+      // Drain: the last load issued into every stage has landed before the CTA
+      // may exit (on the fault-free path they all have by the time consumers
+      // finish; after a failure this bounds the wait for a load left in flight).
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int i = 0; i < 2; ++i) mbar_wait_until(q_full + i, 0, deadline);
+      for (int st = 0; st < NK && st < nk_issued; ++st) {
+        const int last = st + ((nk_issued - 1 - st) / NK) * NK;
+        mbar_wait_until(k_full + st, (last / NK) & 1, deadline);
+      }
+      for (int st = 0; st < NV && st < nv_issued; ++st) {
+        const int last = st + ((nv_issued - 1 - st) / NV) * NV;
+        mbar_wait_until(v_full + st, (last / NV) & 1, deadline);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp walks the schedule (named barriers are warp-aligned); lane 0 issues.
       constexpr uint32_t fmt = FP8 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
-      constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, BM, BN);  // Q, K both K-major
+      constexpr uint32_t idesc_s = I8QK ? make_idesc_s8(BM, BN) : make_idesc(fmt, fmt, 0, BM, BN);  // both K-major
       constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 1, BM, D);   // V MN-major (d contiguous)
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
@@ -289,7 +355,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < D / C::kKStep; ++kk) {
           const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;  // 32 bytes of K per MMA
           const uint64_t ad = smem_desc_sw128(qa + off, 16, 1024), bd = smem_desc_sw128(ka + off, 16, 1024);
-          if constexpr (FP8)
+          if constexpr (I8QK)
+            mma_i8_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          else if constexpr (FP8)
             mma_f8_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           else
             mma_f16_ss(tmem + C::kColS + 128 * i, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
@@ -312,7 +380,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       const bool leader = lane == 0;
       uint64_t* q_in = FP8 ? q_full : q_ready;  // BF16 waits for the in-place rotation
-      bool ok = mbar_wait(q_in, 0, err, kErrTimeout) && mbar_wait(k_full, 0, err, kErrTimeout);
+      bool ok = mbar_wait(q_in, 0, err, kErrTimeout, abort_flag) && mbar_wait(k_full, 0, err, kErrTimeout, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
@@ -321,7 +389,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(s_full);
           mma_commit(k_empty);
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(q_in + 1, 0, err, kErrTimeout));
+        ok = __all_sync(0xffffffffu, mbar_wait(q_in + 1, 0, err, kErrTimeout, abort_flag));
       }
       if (ok) {
         tc_fence_after();
@@ -332,12 +400,16 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
-      for (int j = 1; ok && j <= nkv; ++j) {
+      int j = 1;
+      for (; ok && j <= nkv; ++j) {
         const int jj = j - 1, sv = jj % NV, sk = j % NK;
-        // TMA readiness first, while the softmax warpgroups are still busy
-        ok = mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout);
-        if (ok && j < nkv) ok = mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout);
-        if (!__all_sync(0xffffffffu, ok)) break;
+        // another role gave up: stop issuing.  Then TMA readiness, while the
+        // softmax warpgroups are still busy
+        ok = flag_load(abort_flag) == 0;
+        ok = ok && mbar_wait(v_full + sv, (jj / NV) & 1, err, kErrTimeout, abort_flag);
+        if (ok && j < nkv) ok = mbar_wait(k_full + sk, (j / NK) & 1, err, kErrTimeout, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         constexpr int NKK = BN / C::kKStep, KH = C::kSplitP ? NKK / 2 : 0;
         if constexpr (C::kSplitP) {  // first half of PV_0 while softmax 0 finishes P_0
           named_sync<kBarPHalf + 0, 160>();
@@ -349,13 +421,14 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         if (leader) {
           pv(0, sv, KH > 0 || jj > 0, KH, NKK);
-          mma_commit(pv_done);
+          if (j == nkv) mma_commit(pv_done);  // the epilogue waits for the last PV only
           mma_commit(v_empty + sv);
           if (j < nkv) {
             qk(0, sk);
             mma_commit(s_full);
             mma_commit(k_empty + sk);
           }
+          flag_store(mma_done, j);
         }
         __syncwarp();
         if constexpr (C::kSplitP) {
@@ -368,15 +441,27 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         if (leader) {
           pv(1, sv, KH > 0 || jj > 0, KH, NKK);
-          mma_commit(pv_done + 1);
+          if (j == nkv) mma_commit(pv_done + 1);  // the epilogue waits for the last PV only
           mma_commit(v_empty + sv);
           if (j < nkv) {
             qk(1, sk);
             mma_commit(s_full + 1);
             mma_commit(k_empty + sk);
           }
+          flag_store(mma_done + 4, j);
         }
         __syncwarp();
+      }
+      if (!ok) {
+        // Failure path: the rest of the named-barrier schedule, no MMAs.
+        for (; j <= nkv; ++j) {
+          if constexpr (C::kSplitP) named_sync<kBarPHalf + 0, 160>();
+          named_sync<kBarPReady + 0, 160>();
+          if (leader) flag_store(mma_done, j);
+          if constexpr (C::kSplitP) named_sync<kBarPHalf + 1, 160>();
+          named_sync<kBarPReady + 1, 160>();
+          if (leader) flag_store(mma_done + 4, j);
+        }
       }
    }
   } else {
@@ -388,13 +473,16 @@ __global__ void __launch_bounds__(384, 1)
     // First, while almost nothing is live: the per-tile loop's constants are formed
     // after it, so the preparation's registers cannot push them into local memory
     // (measured: 6 % slower per tile when it ran after them).
+    bool ok = true;
     if constexpr (!FP8) {
       uint64_t* qf = q_full + i;
-      auto wait_tile = [qf, err]() { return mbar_wait(qf, 0, err, kErrTimeout); };
-      rotate_q_tile<D>(sQ + i * C::kTileBytes, out.rope_cos, out.rope_sin, qblk * BM, N, wait_tile);
+      auto wait_tile = [qf, err, abort_flag]() { return mbar_wait(qf, 0, err, kErrTimeout, abort_flag); };
+      ok = __all_sync(0xffffffffu,
+                      rotate_q_tile<D>(sQ + i * C::kTileBytes, out.rope_cos, out.rope_sin, qblk * BM, N, wait_tile));
       // the MMA reads Q through the async proxy: order the generic-proxy writes first
       fence_proxy_async_smem();
-      mbar_arrive(q_ready + i);
+      // only a tile that came is handed on; otherwise the MMA warp's bounded wait gives up
+      if (ok) mbar_arrive(q_ready + i);
     }
     const int row = threadIdx.x & 127;          // TMEM lane = row of the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -445,9 +533,20 @@ __global__ void __launch_bounds__(384, 1)
     };
     float m = -INFINITY;  // running (possibly stale) max of the scaled log2 scores
     float l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, j & 1, err, kErrTimeout));
+    // FP8: the K and V block scales of the next tile, loaded one tile ahead so that
+    // their global-memory latency stays off the per-tile critical path
+    float ksn0 = 1.f, ksn1 = 1.f, vsn0 = 1.f, vsn1 = 1.f;
+    if constexpr (FP8) {
+      ksn0 = ksc[0];
+      vsn0 = vsc[0];
+      if (1 < nk) {
+        ksn1 = ksc[1];
+        vsn1 = vsc[1];
+      }
+    }
+    int j = 0;
+    for (; ok && j < nkv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full + i, j & 1, err, kErrTimeout, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[BN];
@@ -455,6 +554,10 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_wait_ld();
       reg_fence(s);
+      if constexpr (I8QK) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = s32_biased_f32(s[c]);
+      }
       const int kv0 = j * BN;
       if (kv0 + BN > N) {
 #pragma unroll
@@ -464,24 +567,32 @@ __global__ void __launch_bounds__(384, 1)
       // per-64-key-half score multipliers (both equal for BF16)
       float c0 = sl2, c1 = sl2, f0 = 1.f, f1 = 1.f;
       if constexpr (FP8) {
-        const int kb0 = 2 * j, kb1 = 2 * j + 1;
-        c0 = qs * ksc[kb0];
-        c1 = kb1 < nk ? qs * ksc[kb1] : 1.f;  // past the end every key is -inf; keep -inf * c1 = -inf
-        f0 = vsc[kb0] * vfold;
-        f1 = kb1 < nk ? vsc[kb1] * vfold : 1.f;  // past the end every p is 0 anyway
+        // a half past the end keeps 1: its keys are -inf (-inf * c1 = -inf) and its p are 0
+        c0 = qs * ksn0;
+        c1 = qs * ksn1;
+        f0 = vsn0 * vfold;
+        f1 = vsn1 * vfold;
+        const int kb0 = 2 * j + 2, kb1 = 2 * j + 3;  // the next tile's blocks
+        ksn0 = kb0 < nk ? ksc[kb0] : 1.f;
+        vsn0 = kb0 < nk ? vsc[kb0] : 1.f;
+        ksn1 = kb1 < nk ? ksc[kb1] : 1.f;
+        vsn1 = kb1 < nk ? vsc[kb1] : 1.f;
       }
-      // row max: two 3-input max chains per 64-key half
-      float ma0 = __uint_as_float(s[0]), ma1 = __uint_as_float(s[1]);
-      float mb0 = __uint_as_float(s[64]), mb1 = __uint_as_float(s[65]);
+      // row max: two 3-input max chains per 64-key half (keys 0..3 of the half start
+      // the chains, then four keys per step up to key 63 of the half)
+      float ma0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
+      float ma1 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
+      float mb0 = fmaxf(__uint_as_float(s[64]), __uint_as_float(s[65]));
+      float mb1 = fmaxf(__uint_as_float(s[66]), __uint_as_float(s[67]));
 #pragma unroll
-      for (int c = 2; c < 64; c += 4) {
+      for (int c = 4; c < 64; c += 4) {
         ma0 = fmax3(ma0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
         ma1 = fmax3(ma1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
         mb0 = fmax3(mb0, __uint_as_float(s[64 + c]), __uint_as_float(s[64 + c + 1]));
         mb1 = fmax3(mb1, __uint_as_float(s[64 + c + 2]), __uint_as_float(s[64 + c + 3]));
       }
-      const float mx0 = fmaxf(ma0, ma1);
-      const float mx1 = fmaxf(mb0, mb1);
+      const float mx0 = fmaxf(ma0, ma1) - (I8QK ? kI8Bias : 0.f);  // exact: both within [2^23, 2^24)
+      const float mx1 = fmaxf(mb0, mb1) - (I8QK ? kI8Bias : 0.f);
       // the first key of a tile is always in range; a half past the end is all -inf
       const float m_tile = fmaxf(mx0 * c0, kv0 + 64 < N ? mx1 * c1 : -INFINITY);
       const bool grow = __any_sync(0xffffffffu, m_tile > m + C::kRescaleLog2);
@@ -502,7 +613,10 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t nm2 = f2(-m_new, -m_new);
       // FP8: the V block scale of each 64-key half enters as an exponent offset,
       // p * f = 2^(x - m + log2 f), which saves a multiply per element.
-      const float lf0 = FP8 ? lg2(f0) - m_new : 0.f, lf1 = FP8 ? lg2(f1) - m_new : 0.f;
+      // I8QK: the scores in s are biased by kI8Bias; the bias times the half's
+      // multiplier comes off here, once per tile, so x = s c + lf stays one FMA.
+      const float lf0 = FP8 ? lg2(f0) - m_new - (I8QK ? kI8Bias * c0 : 0.f) : 0.f;
+      const float lf1 = FP8 ? lg2(f1) - m_new - (I8QK ? kI8Bias * c1 : 0.f) : 0.f;
       const uint64_t nmA = f2(lf0, lf0), nmB = f2(lf1, lf1);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       constexpr int kPRegs = FP8 ? 32 : 64;  // packed P of the whole row
@@ -515,10 +629,18 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int k0 = 32 * q + 4 * e;
-            float x0, x1, x2, x3;
-            f2_split(ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), cq, nmq), x0, x1);
-            f2_split(ffma2(f2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), cq, nmq), x2, x3);
-            const float a = ex2(x0), bq = ex2(x1), cc = ex2(x2), dd = ex2(x3);
+            const uint64_t xa = ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), cq, nmq);
+            const uint64_t xb = ffma2(f2(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), cq, nmq);
+            float a, bq, cc, dd;
+            if ((C::kPolyMask >> (8 * (q & 1) + e)) & 1u) {  // on the FMA pipe
+              ex2_poly_pair(xa, a, bq);
+              ex2_poly_pair(xb, cc, dd);
+            } else {
+              float x0, x1, x2, x3;
+              f2_split(xa, x0, x1);
+              f2_split(xb, x2, x3);
+              a = ex2(x0), bq = ex2(x1), cc = ex2(x2), dd = ex2(x3);
+            }
             // row sums per 64-key half (each carries its own V block scale)
             acc[2 * (q >> 1)] = fadd2(acc[2 * (q >> 1)], f2(a, bq));
             acc[2 * (q >> 1) + 1] = fadd2(acc[2 * (q >> 1) + 1], f2(cc, dd));
@@ -528,10 +650,17 @@ __global__ void __launch_bounds__(384, 1)
         } else {  // 32 keys -> 16 columns of 2 bf16
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float x, y;
-            f2_split(ffma2(f2(__uint_as_float(s[32 * q + 2 * e]), __uint_as_float(s[32 * q + 2 * e + 1])), cq, nm2), x,
-                     y);
-            const float p0 = ex2(x), p1 = ex2(y);
+            const uint64_t xy =
+                ffma2(f2(__uint_as_float(s[32 * q + 2 * e]), __uint_as_float(s[32 * q + 2 * e + 1])), cq, nm2);
+            float p0, p1;
+            if ((C::kPolyMask >> e) & 1u) {  // on the FMA pipe
+              ex2_poly_pair(xy, p0, p1);
+            } else {
+              float x, y;
+              f2_split(xy, x, y);
+              p0 = ex2(x);
+              p1 = ex2(y);
+            }
             acc[e & 3] = fadd2(acc[e & 3], f2(p0, p1));
             p[16 * q + e] = pack_bf16x2(p0, p1);
           }
@@ -569,8 +698,38 @@ __global__ void __launch_bounds__(384, 1)
       }
       m = m_new;
     }
+    if (!ok) {
+      // Failure path: the rest of this warpgroup's named-barrier schedule (tiles j..nkv-1)
+      // without the work between, so the MMA warp and the other warpgroup are never
+      // left waiting on an arrival from here.  Each arrival waits (bounded) until the
+      // partner has passed the previous generation of that barrier.
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      const uint32_t my_mma_done = mma_done + 4 * i;
+      for (; j < nkv; ++j) {
+        if constexpr (C::kPingPong) {
+          if (i == 1) named_sync<kBarTurn + 1, 256>();
+          else if (j > 0) named_sync<kBarTurn + 0, 256>();
+        }
+        if (!warp_wait_flag_ge(my_mma_done, j, deadline)) break;
+        if constexpr (C::kSplitP) {
+          if (i == 0) named_arrive<kBarPHalf + 0, 160>();
+          else named_arrive<kBarPHalf + 1, 160>();
+        }
+        if constexpr (C::kPingPong) {
+          if (i == 0) {
+            if (!warp_wait_flag_ge(mma_done + 4, j, deadline)) break;  // warpgroup 1 passed Turn_1(j-1)
+            named_arrive<kBarTurn + 1, 256>();
+          } else if (j + 1 < nkv) {
+            if (!warp_wait_flag_ge(mma_done, j + 1, deadline)) break;  // warpgroup 0 passed Turn_0(j-1)
+            named_arrive<kBarTurn + 0, 256>();
+          }
+        }
+        if (i == 0) named_arrive<kBarPReady + 0, 160>();
+        else named_arrive<kBarPReady + 1, 160>();
+      }
+    }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, (nkv - 1) & 1, err, kErrTimeout));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, 0, err, kErrTimeout, abort_flag));
     if (ok) {
       tc_fence_after();
       const float fin = fin_scale / l;
@@ -602,18 +761,26 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 9) {
     __syncwarp();
     tc_fence_after();
+    if (flag_load(abort_flag) != 0) {
+      // after a failure nobody waited for the last MMAs: wait (bounded) until every
+      // MMA issued has completed, so that TMEM is not released under a running one
+      if (lane == 0) mma_commit(mma_drain);
+      __syncwarp();
+      mbar_wait_until(mma_drain, 0, globaltimer_ns() + kWaitLimitNs);
+    }
     tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
-template <bool FP8, int D>
+template <bool FP8, int D, bool I8QK = false>
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
                         const AttnScales& sc, int B, int H, cudaStream_t stream) {
   constexpr int smem = AttnCfg<FP8, D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<FP8, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_kernel<FP8, D, I8QK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((out.N + 255) / 256, H, B);
-  attn_kernel<FP8, D><<<grid, AttnCfg<FP8, D>::kThreads, smem, stream>>>(tq, tk, tv, out, sc);
+  attn_kernel<FP8, D, I8QK><<<grid, AttnCfg<FP8, D>::kThreads, smem, stream>>>(tq, tk, tv, out, sc);
   return cudaGetLastError();
 }
 

@@ -269,10 +269,14 @@ size_t dit_attn_fp8_workspace_bytes(int B, int H, int N, int d, int q_block, int
          align256(bh * 4) + align256(bh * dit::kFp8MeanChunks * d * 4);
 }
 
-dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
-                        const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
-                        const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
-                        int smooth_k, void* workspace, size_t workspace_bytes, dit_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+dit_status attn_fp8_impl(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                         const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
+                         int smooth_k, void* workspace, size_t workspace_bytes, int qk_int8, dit_stream_t stream) {
   if (!q || !k || !v || !o || !sq || !sk || !sv || !so) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return DIT_ERR_INVALID_ARG;
@@ -298,6 +302,7 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   }
   p.cos_tab = rope_cos; p.sin_tab = rope_sin;
   p.B = B; p.H = H; p.N = N; p.d = d; p.q_block = q_block; p.kv_block = kv_block; p.smooth_k = smooth_k != 0;
+  p.qk_int8 = qk_int8;
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t el = bh * N * d;
   const size_t nq = (N + q_block - 1) / q_block, nk = (N + kv_block - 1) / kv_block;
@@ -315,7 +320,7 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
   // Every map is built before the first launch, so an error return leaves nothing enqueued.
   CUtensorMap tq, tk, tv;
-  // e4m3: one 128-byte row holds all d = 128 channels of a token.
+  // 8-bit codes (e4m3, or int8 for Q and K): one 128-byte row holds all d = 128 channels of a token.
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.q8, B, H, N, d, cs, 128, 128) ||
       !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.k8, B, H, N, d, cs, 128, dit::kAttnBlockN) ||
       !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.v8, B, H, N, d, cs, 128, dit::kAttnBlockN))
@@ -331,6 +336,27 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
   out.rope_cos = nullptr;  // Q arrives rotated and quantised from the prologue
   out.rope_sin = nullptr;
   return launch_status(dit::launch_attn_fp8(tq, tk, tv, out, p, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                        const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                        const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
+                        int smooth_k, void* workspace, size_t workspace_bytes, dit_stream_t stream) {
+  return attn_fp8_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, q_block, kv_block,
+                       smooth_k, workspace, workspace_bytes, 0, stream);
+}
+
+dit_status dit_attn_fp8_i8qk(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                             const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
+                             const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block,
+                             int kv_block, int smooth_k, void* workspace, size_t workspace_bytes,
+                             dit_stream_t stream) {
+  return attn_fp8_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, q_block, kv_block,
+                       smooth_k, workspace, workspace_bytes, 1, stream);
 }
 
 size_t fbcache_gate_workspace_bytes(int64_t n) {
@@ -361,6 +387,16 @@ dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int64_t n, d
   if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
   return launch_status(dit::launch_gate_sums(r_cur, r_prev, n, sums_out, static_cast<double*>(workspace),
                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dit_status fbcache_gate_ref_update(const void* r_cur, void* r_ref, int64_t n, const int32_t* skip,
+                                   dit_stream_t stream) {
+  if (!r_cur || !r_ref || n < 1) return DIT_ERR_INVALID_ARG;
+  if (!aligned16(r_cur) || !aligned16(r_ref) || !aligned4(skip)) return DIT_ERR_ALIGNMENT;
+  if (r_cur == r_ref) return DIT_ERR_INVALID_ARG;
+  const DeviceState* ds = device_state();
+  if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
+  return launch_status(dit::launch_gate_ref_update(r_cur, r_ref, n, skip, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,

@@ -72,11 +72,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Bounded: after
-// kWaitLimitNs of wall time it records `code` in the error word and returns
-// false, so that a lost arrival never hangs the GPU.
+// kWaitLimitNs of wall time it records `code` in the error word, raises the
+// CTA's abort flag (when one is given) and returns false, so that a lost
+// arrival never hangs the GPU.  With an abort flag it also gives up, without
+// recording anything, as soon as another role of the CTA has raised the flag:
+// the arrival it waits for may never come once a partner has stopped.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+// A flag word in shared memory, addressed by its 32-bit shared-window address
+// (one register, where a generic pointer takes two).
+// (volatile asm: kept in program order with the barrier and wait instructions,
+// which are volatile asm too; no compiler memory barrier is needed around them.)
+__device__ __forceinline__ int flag_load(uint32_t a) {
+  int v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void flag_store(uint32_t a, int v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(a), "r"(v));
+}
+
+// Warp-uniform wait until the shared flag at `a` is at least `target`, or until
+// the %globaltimer time `deadline_ns`; true when the flag got there.
+__device__ __forceinline__ bool warp_wait_flag_ge(uint32_t a, int target, uint64_t deadline_ns) {
+  while (true) {
+    if (__all_sync(0xffffffffu, flag_load(a) >= target)) return true;
+    if (__any_sync(0xffffffffu, globaltimer_ns() > deadline_ns)) return false;
+  }
+}
+
+// abort_flag: shared-window address of the CTA's abort flag, or 0 for none.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code,
+                                          uint32_t abort_flag = 0) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -84,10 +111,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
+    if (abort_flag != 0 && flag_load(abort_flag) != 0) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       set_error(err, code);
+      if (abort_flag != 0) flag_store(abort_flag, 1);
       return false;
     }
+  }
+}
+
+// Waits for the phase with the given parity until the absolute %globaltimer
+// time `deadline_ns`; true when the phase completed.  Records nothing.
+__device__ __forceinline__ bool mbar_wait_until(uint64_t* bar, uint32_t parity, uint64_t deadline_ns) {
+  const uint32_t a = smem_u32(bar);
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(a, parity)) return true;
+    if (globaltimer_ns() > deadline_ns) return false;
   }
 }
 
@@ -225,6 +266,16 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// kind::i8 form (s8 x s8 -> s32), both operands in shared memory.
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every MMA issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -259,6 +310,12 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt
                                                   uint32_t N) {
   return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (0u << 15) | (b_mn_major << 16) | ((N >> 3) << 17) |
          ((M >> 4) << 24);
+}
+
+// Instruction descriptor for dense kind::i8 MMA: signed 8-bit A and B (both
+// K-major), s32 accumulation ([4,6) D format 2 = s32; [7,10), [10,13) 1 = signed).
+__host__ __device__ constexpr uint32_t make_idesc_s8(uint32_t M, uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // Named CTA barriers (ids 1..15; 0 is __syncthreads).  `count` threads take part
@@ -319,6 +376,43 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x for a pair of floats on the FMA and integer pipes instead of the MUFU unit
+// (which executes ex2 at a quarter of the FMA rate and is the softmax's
+// bottleneck).  Cody-Waite split x = j + f, j = round(x), f in [-0.5, 0.5];
+// 2^f by a cubic fitted for relative error on that interval (max 7.5e-5, far
+// below the bf16 / e4m3 rounding of P that follows); 2^j added to the exponent
+// field.  j comes from the float sum x + 1.5 * 2^23 (whose low bits are round(x)
+// when |x| < 2^22); the bias bits vanish in the shift by 23.  x is clamped at
+// -126, below which the result is 2^-126 or less instead of 2^x (the exponent
+// field must not go below zero).
+__device__ __forceinline__ void ex2_poly_pair(uint64_t x2, float& a, float& b) {
+  constexpr float kBias = 12582912.0f;  // 1.5 * 2^23
+  float x0, x1;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(x0), "=f"(x1) : "l"(x2));
+  uint64_t xc;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(xc) : "f"(fmaxf(x0, -126.f)), "f"(fmaxf(x1, -126.f)));
+  uint64_t bias2, nbias2, neg1, c3, c2, c1, c0;
+  asm("mov.b64 %0, {%1,%1};" : "=l"(bias2) : "f"(kBias));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(nbias2) : "f"(-kBias));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(neg1) : "f"(-1.f));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c3) : "f"(0.055171605f));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c2) : "f"(0.24261111f));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c1) : "f"(0.69326097f));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c0) : "f"(0.99992806f));
+  uint64_t t, jf, fr, p;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xc), "l"(bias2));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(jf) : "l"(t), "l"(nbias2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(fr) : "l"(jf), "l"(neg1), "l"(xc));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(fr), "l"(c3), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(fr), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(fr), "l"(c0));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0,%1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0,%1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  a = __uint_as_float(p0 + (t0 << 23));
+  b = __uint_as_float(p1 + (t1 << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -43,6 +43,10 @@ cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* su
 cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
                                  cudaStream_t stream);
 
+// ref = cur (n bf16 elements, 16-byte aligned) unless skip is non-null and *skip != 0
+// at execution time.
+cudaError_t launch_gate_ref_update(const void* cur, void* ref, int64_t n, const int32_t* skip, cudaStream_t stream);
+
 // Output description shared by the attention kernels.
 struct AttnOut {
   void* o;          // bf16 [B,H,N,d]
@@ -73,6 +77,9 @@ struct Fp8Prep {
   int B, H, N, d;
   int q_block, kv_block;
   int smooth_k;
+  // 0: Q and K in e4m3 (scale amax/448); 1: Q and K in symmetric int8 (scale
+  // amax/127, for the 8-bit integer Q.K^T).  V is e4m3 either way.
+  int qk_int8;
   // workspace carve-out
   uint8_t* q8;      // e4m3 [B,H,N,d]
   uint8_t* k8;      // e4m3 [B,H,N,d]
@@ -92,6 +99,7 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream);
 // One thread waits (bounded) on an mbarrier nothing arrives on: records kErrTimeout.
 cudaError_t launch_selftest_wait(int* err, cudaStream_t stream);
 
+// FP8 attention over the prologue's output; p.qk_int8 selects the Q.K^T form.
 cudaError_t launch_attn_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnOut& out,
                             const Fp8Prep& p, cudaStream_t stream);
 

@@ -16,6 +16,10 @@
 //   and K in fp32, subtract the K mean,
 //   block amax, scale and cast to e4m3; write the scales.  Streams 6 B/element
 //   in (bf16 Q, K, V) and 3 B/element out; HBM-bound.
+// With qk_int8 (the 8-bit integer Q.K^T of SageAttention, the quantised
+// attention the same ledger row names), Q and K are cast instead to symmetric
+// int8: scale amax/127 per block, round to nearest even, within +-127; V stays
+// e4m3.
 #include <cuda_bf16.h>
 
 #include "dit_device.cuh"
@@ -115,12 +119,30 @@ __global__ void __launch_bounds__(128) kmean_finalize(Fp8Prep p, const float* __
   p.k_mean[bh * 128 + c] = p.smooth_k ? sum / static_cast<float>(p.N) : 0.f;
 }
 
+// Eight floats times inv (within [-127, 127]) -> eight int8 (two's complement),
+// rounded to nearest even, in token-row byte order.  fma(x, inv, 1.5 * 2^23)
+// rounds x * inv once to an integer (the float's unit in the last place is 1
+// there), and the float's low byte is then that integer modulo 256.
+__device__ __forceinline__ uint32_t s8_bits(float x, float inv) {
+  return __float_as_uint(__fmaf_rn(x, inv, 12582912.0f));
+}
+__device__ __forceinline__ uint32_t cvt_s8x4(const float* x, float inv) {
+  // byte_perm selector nibbles pick bytes of {y:x}: low bytes of the four codes, in order
+  const uint32_t ab = __byte_perm(s8_bits(x[0], inv), s8_bits(x[1], inv), 0x0040);
+  const uint32_t cd = __byte_perm(s8_bits(x[2], inv), s8_bits(x[3], inv), 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
+__device__ __forceinline__ uint2 cvt_s8x8(const float (&x)[8], float inv) {
+  return make_uint2(cvt_s8x4(x, inv), cvt_s8x4(x + 4, inv));
+}
+
 // Quantises one 128-token block of one tensor held as 8 chunks per thread:
 // thread t owns channel chunk (t % 16) of tokens t/16 + 16 i, i = 0..7.  With
 // two_blocks the first four tokens of a thread lie in the first 64-token block.
+// int8: symmetric int8 codes and scales amax/127 instead of e4m3 and amax/448.
 __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks, int n_base, int N,
                                               uint8_t* __restrict__ dst, int cc, int tl, float* red, float* sc_out0,
-                                              float* sc_out1, float* vmax) {
+                                              float* sc_out1, float* vmax, bool int8 = false) {
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i)
@@ -133,10 +155,11 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
     }
   a0 = block_max(a0, red);
   if (two_blocks) a1 = block_max(a1, red + 8);
-  const float s0 = a0 > 0.f ? a0 / 448.f : 1.f;
-  const float s1 = a1 > 0.f ? a1 / 448.f : 1.f;
-  const float inv0 = a0 > 0.f ? 448.f / a0 : 1.f;
-  const float inv1 = a1 > 0.f ? 448.f / a1 : 1.f;
+  const float qmax = int8 ? 127.f : 448.f;
+  const float s0 = a0 > 0.f ? a0 / qmax : 1.f;
+  const float s1 = a1 > 0.f ? a1 / qmax : 1.f;
+  const float inv0 = a0 > 0.f ? qmax / a0 : 1.f;
+  const float inv1 = a1 > 0.f ? qmax / a1 : 1.f;
   if (threadIdx.x == 0) {
     *sc_out0 = s0;
     if (two_blocks) *sc_out1 = s1;
@@ -152,8 +175,12 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
     if (n >= N) continue;
     const float inv = (i < 4 || !two_blocks) ? inv0 : inv1;
     uint2 w;
-    w.x = cvt_e4m3x2(x[i][0] * inv, x[i][1] * inv) | (cvt_e4m3x2(x[i][2] * inv, x[i][3] * inv) << 16);
-    w.y = cvt_e4m3x2(x[i][4] * inv, x[i][5] * inv) | (cvt_e4m3x2(x[i][6] * inv, x[i][7] * inv) << 16);
+    if (int8) {
+      w = cvt_s8x8(x[i], inv);
+    } else {
+      w.x = cvt_e4m3x2(x[i][0] * inv, x[i][1] * inv) | (cvt_e4m3x2(x[i][2] * inv, x[i][3] * inv) << 16);
+      w.y = cvt_e4m3x2(x[i][4] * inv, x[i][5] * inv) | (cvt_e4m3x2(x[i][6] * inv, x[i][7] * inv) << 16);
+    }
     *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(n) * 128 + cc * 8) = w;
   }
 }
@@ -162,6 +189,8 @@ __device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks,
 // 128-token block, rotated), 1 quantises K (two 64-token blocks, rotated and
 // smoothed), 2 quantises V (two 64-token blocks).  Every thread issues its eight
 // 16-byte loads before any reduction, so each CTA keeps 32 KB in flight.
+// INT8: Q and K as symmetric int8 (the integer Q.K^T form), V as e4m3.
+template <bool INT8>
 __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
   const int blk = blockIdx.x;  // 128-token block
   const int bh = blockIdx.y;
@@ -203,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
       for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
   }
   if (which == 0) {
-    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr);
+    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr,
+                  INT8);
     return;
   }
   if (which == 1) {
@@ -217,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
       }
     }
     float* s1 = (2 * blk + 1 < nk) ? p.k_scale + bh * nk + 2 * blk + 1 : &unused_scale;
-    quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr);
+    quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr,
+                  INT8);
     return;
   }
   float* s1 = (2 * blk + 1 < nk) ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
@@ -237,7 +268,10 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((p.N + 127) / 128, p.B * p.H, 3);
-  quantize_qkv<<<g2, kThreads, 0, stream>>>(p);
+  if (p.qk_int8)
+    quantize_qkv<true><<<g2, kThreads, 0, stream>>>(p);
+  else
+    quantize_qkv<false><<<g2, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -16,6 +16,7 @@
 // the caller) and gate_finalize takes the decision from the summed totals.
 #include <cuda_bf16.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "dit.h"
@@ -182,6 +183,49 @@ cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel
   return cudaGetLastError();
 }
 
+// Reference residual of the gate's policies: r_ref = r_cur, unless the flag says
+// the step was skipped (then the reference stays the last computed step's).
+// Every CTA reads the flag once and returns at once when it is set; otherwise a
+// grid-strided 16-byte copy with four loads in flight per thread (HBM-bound,
+// 4 bytes moved per element).
+__global__ void __launch_bounds__(kGateThreads) gate_ref_update(const uint4* __restrict__ cur, uint4* __restrict__ ref,
+                                                                int64_t n8, const int32_t* __restrict__ skip) {
+  if (skip != nullptr && *skip != 0) return;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n8; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldcs(cur + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ref[i + u * stride] = v[u];
+  }
+  for (; i < n8; i += stride) ref[i] = __ldcs(cur + i);
+}
+
+__global__ void gate_ref_update_tail(const __nv_bfloat16* __restrict__ cur, __nv_bfloat16* __restrict__ ref,
+                                     int64_t from, int64_t n, const int32_t* __restrict__ skip) {
+  if (skip != nullptr && *skip != 0) return;
+  const int64_t t = from + threadIdx.x;
+  if (t < n) ref[t] = cur[t];
+}
+
+cudaError_t launch_gate_ref_update(const void* cur, void* ref, int64_t n, const int32_t* skip, cudaStream_t stream) {
+  const int64_t n8 = n / 8;
+  if (n8 > 0) {
+    gate_ref_update<<<gate_num_ctas(n), kGateThreads, 0, stream>>>(static_cast<const uint4*>(cur),
+                                                                   static_cast<uint4*>(ref), n8, skip);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (n - n8 * 8 > 0) {
+    gate_ref_update_tail<<<1, 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(cur),
+                                                static_cast<__nv_bfloat16*>(ref), n8 * 8, n, skip);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
 }  // namespace dit
 
 // ---------------------------------------------------------------------------
@@ -236,7 +280,7 @@ double* noalloc_scratch(dit_status* st) {
 extern "C" DIT_API dit_status fbcache_gate_noalloc(const void* r_cur, const void* r_prev, int64_t n, float threshold,
                                                    float* rel_out, int32_t* skip_out, dit_stream_t stream) {
   if (!r_cur || !r_prev || !rel_out || !skip_out || n < 1) return DIT_ERR_INVALID_ARG;
-  if (!(threshold == threshold) || threshold > 3.4e38f || threshold < -3.4e38f) return DIT_ERR_INVALID_ARG;
+  if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(r_cur) & 15u) || (reinterpret_cast<uintptr_t>(r_prev) & 15u) ||
       (reinterpret_cast<uintptr_t>(rel_out) & 3u) || (reinterpret_cast<uintptr_t>(skip_out) & 3u))
     return DIT_ERR_ALIGNMENT;

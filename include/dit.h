@@ -13,6 +13,8 @@
  *                    Same page (cuDNN FP8 attention against VANILLA BF16) and
  *                    "vflash / Optimization ledger", table "Accepted or
  *                    exposed" (SageAttention2, a quantised attention).
+ *   dit_attn_fp8_i8qk  the same with Q and K as symmetric int8 (8-bit integer
+ *                    Q.K^T, e4m3 P.V): the SageAttention2 row of that table.
  *   dit_rope_tables  cos/sin tables of the multi-axis rotary embedding.
  *   rope_apply       rotary embedding applied to a [B,H,N,d] tensor.
  *                    "vflash / Optimization ledger", row "strict Triton RoPE".
@@ -173,6 +175,25 @@ DIT_API dit_status dit_attn_fp8(const void* q, const void* k, const void* v, voi
                         const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
                         int smooth_k, void* workspace, size_t workspace_bytes, dit_stream_t stream);
 
+/* FP8 attention with an 8-bit integer Q.K^T: the quantised attention of
+ * "vflash / Optimization ledger", table "Accepted or exposed", SageAttention2
+ * row (8-bit integer Q.K^T, FP8 P.V).  As dit_attn_fp8 except that the rotated
+ * Q and the rotated, smoothed K are quantised to symmetric int8 (one fp32
+ * scale amax/127 per block of q_block or kv_block tokens, round to nearest
+ * even, within +-127) and S = Q8 K8^T accumulates exactly in int32 on the
+ * tensor cores (kind::i8) before it is scaled by sQ * sK * softmax_scale.  V,
+ * P and everything after the scores are as in dit_attn_fp8.  Where a few
+ * channels of Q and K carry outliers, the integer codes keep the large
+ * products to within 1/254 of the block maximum where e4m3 keeps 1/16 of
+ * each product, so the result stays much closer to exact attention.  The
+ * workspace layout and size are dit_attn_fp8's
+ * (dit_attn_fp8_workspace_bytes); same supported sizes and errors. */
+DIT_API dit_status dit_attn_fp8_i8qk(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                                     const int64_t sq[3], const int64_t sk[3], const int64_t sv[3],
+                                     const int64_t so[3], const float* rope_cos, const float* rope_sin,
+                                     float softmax_scale, int q_block, int kv_block, int smooth_k, void* workspace,
+                                     size_t workspace_bytes, dit_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* First-Block-Cache gate                                                    */
 /* ------------------------------------------------------------------------ */
@@ -201,6 +222,19 @@ DIT_API dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int6
  * skip = rel < threshold, written to rel_out / skip_out (device). */
 DIT_API dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
                                          dit_stream_t stream);
+
+/* The gate's reference residual, for the two reference policies of the step
+ * cache (unsloth studio commit "core/inference/diffusion.py", "Add opt-in step
+ * caching (First-Block-Cache)": the threshold knob; which step the residual is
+ * compared with is left open): r_ref = r_cur over n contiguous bf16 elements,
+ * unless skip is non-NULL and *skip != 0 when the copy runs, in which case
+ * r_ref is left as it is.  Called after fbcache_gate with that call's skip_out,
+ * it keeps r_ref at the residual of the last step whose remaining blocks ran
+ * ("last computed" policy) without a host read; with skip NULL it copies
+ * unconditionally (the "consecutive" policy, previous step).  r_cur, r_ref
+ * 16-byte aligned and distinct, skip 4-byte aligned; n >= 1. */
+DIT_API dit_status fbcache_gate_ref_update(const void* r_cur, void* r_ref, int64_t n, const int32_t* skip,
+                                           dit_stream_t stream);
 
 /* fbcache_gate without a workspace argument (the pages have no counterpart:
  * this is a convenience of this library).  For callers that cannot give the

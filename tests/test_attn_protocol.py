@@ -19,21 +19,32 @@ Semantics modelled:
   arrives on its mbarrier once every MMA issued before it has completed; an
   issued MMA may read or write its operands at any moment until it completes.
 * TMA loads land in any order; each arrives on its stage's mbarrier.
-* A named barrier completes when its thread count has arrived; a second
-  arrival by the same role within one generation is an error (the hardware
-  would merge it into the current generation).
+* A named barrier counts arrivals warp by warp (32 threads each); a generation
+  completes the moment its count is reached and the count starts again from
+  zero, so arrivals made ahead of a syncing partner are carried into the next
+  generation as on the hardware.  A second arrival by the same role within one
+  generation is an error on the fault-free path.
 
 Checks: no deadlock; every role finishes; an MMA reads the K/V tile, the Q tile
 (rotated, for BF16) and the half of P it was issued for; no TMA load lands in a
 stage an issued MMA still reads; the softmax reads S and writes P only while no
 issued MMA touches that half of the buffer; O is rescaled and read only while
-no PV into it is outstanding.  Planted protocol mistakes (negative controls)
-must each be caught.
+no PV into it is outstanding; nothing is in flight when the CTA ends.  Planted
+protocol mistakes (negative controls) must each be caught.
 
-Faults: a load or an arrival can be made to never come; the bounded mbarrier
-waits then time out in every order the model can reach, and the tests record
-which losses end every role (the kernel reports DIT_ERR_TIMEOUT and exits) and
-which leave a role at a named barrier, which cannot time out.
+Failure path (as in the kernel): every mbarrier wait is bounded; the first one
+that gives up raises the CTA's abort flag, after which every other bounded wait
+gives up as well.  A role that gives up performs the rest of its named-barrier
+schedule without the work between (the MMA warp its syncs, a softmax
+warpgroup its arrivals and ping-pong turns), so no partner is left on a named
+barrier, which cannot time out.  The BF16 softmax hands its Q tile on only when
+the tile came; the producer waits, bounded, for the last load it issued into
+every stage before it leaves; after a failure the MMA thread waits, bounded,
+for its own MMAs before TMEM is released.  A fault is a load or an arrival that
+never comes: each one, in every configuration, must end every role.  A softmax
+warpgroup is modelled as one role: its four warps each take the same decision
+at every bounded wait or, where they differ, each completes the same schedule
+of named-barrier operations, which is what the dry schedule guarantees.
 """
 import random
 
@@ -55,19 +66,26 @@ class MBar:
 
 
 class Named:
+    """A named barrier of `count` threads: arrivals are counted warp by warp and a
+    generation completes the moment the count is reached."""
+
     def __init__(self, name, count, errors):
         self.name, self.count, self.errors = name, count, errors
         self.arrived, self.gen, self.who = 0, 0, set()
+        self.strict = True  # fault-free runs: no role arrives twice in one generation
 
     def arrive(self, who, n):
-        if who in self.who:
+        """Arrive with n threads (n/32 warps); returns the generation of the last warp."""
+        if who in self.who and self.strict:
             self.errors.append(f"{who} arrives twice at {self.name} in generation {self.gen}")
         self.who.add(who)
-        self.arrived += n
-        if self.arrived > self.count:
-            self.errors.append(f"{self.name}: {self.arrived} arrivals for a count of {self.count}")
-        if self.arrived >= self.count:
-            self.arrived, self.gen, self.who = 0, self.gen + 1, set()
+        g = self.gen
+        for _ in range(n // 32):
+            g = self.gen
+            self.arrived += 32
+            if self.arrived == self.count:
+                self.arrived, self.gen, self.who = 0, self.gen + 1, set()
+        return g
 
 
 CONFIGS = {
@@ -77,23 +95,16 @@ CONFIGS = {
 }
 
 
-def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, report=None):
+def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
     """Run one random interleaving; returns (errors, finished, timeouts).  With a
-    fault injected the result is already invalid once a wait has timed out, so
+    fault injected the result is already invalid once a wait has given up, so
     data hazards no longer stop the run and `errors` holds only a hang.
 
-    fixes: the two failure-path changes planned for the kernel -- the rotating
-    warpgroup arrives on q_ready only when its Q tile came (and otherwise skips
-    its tile loop), and the producer waits, bounded, for the last load it issued
-    into every stage before it leaves.  A lost load is modelled as stalled: issued
-    and in flight, never landing.  report: a dict that receives the loads still in
-    flight when every role has ended and the stages whose drain wait gave up.
-
     lost: a fault to inject -- ("load", kind, tile) for a TMA load that never
-    lands, or ("commit", barrier name, index, nth) for a commit arrival that
-    never comes.  Without a fault no wait may time out; with one, a role whose
-    bounded mbarrier wait cannot complete times out (returns false, as the
-    kernel's mbar_wait does after its limit) and takes the kernel's exit path.
+    lands (issued and in flight), or ("commit", barrier name, index, nth) for a
+    commit arrival that never comes.  Without a fault no wait may give up.
+    report: a dict that receives the loads still in flight when every role has
+    ended, the stages whose drain wait gave up, and whether the abort flag rose.
     """
     rng = random.Random(seed)
     split = pingpong = not fp8
@@ -110,6 +121,11 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
     p_ready = [Named(f"PReady{i}", 160, errors) for i in range(2)]
     p_half = [Named(f"PHalf{i}", 160, errors) for i in range(2)]
     turn = [Named(f"Turn{i}", 256, errors) for i in range(2)]
+    if lost is not None:
+        for b in p_ready + p_half + turn:
+            b.strict = False
+    abort = [False]
+    mma_done = [0, 0]     # PReady_i generations the MMA warp has passed (published after each)
 
     qstate = ["none", "none"]
     kstage, vstage = {}, {}
@@ -183,9 +199,15 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
         full[slot].arrive()
 
     # ------------------------------------------------------------------ roles
-    # A role yields ("mbar", pred) for a bounded mbarrier wait (sent back True when
-    # it completes, False when it times out) or a bare predicate for a wait that
-    # cannot time out (named barriers) or a plain scheduling point.
+    # A role yields ("mbar", pred) for a bounded, abort-aware mbarrier wait (sent
+    # back True when it completes, False when it gives up: on its own limit, which
+    # raises the abort flag, or once the flag is up), ("deadline", pred) for a
+    # bounded wait that ignores the flag (the drains), or a bare predicate for a
+    # wait that cannot time out (named barriers) or a plain scheduling point.
+    def named_sync(bar, who, n):
+        g = bar.arrive(who, n)
+        return lambda: bar.gen > g
+
     def producer():
         for i in range(2):
             load("Q", i, i)  # Q tile i (the tile index names which Q load a fault drops)
@@ -203,21 +225,18 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
                     break
             load("V", sv, j)
             nv_issued += 1
-        if fixes:  # drain: the last load issued into each stage has landed (phase index = tile // ring)
-            for i in range(2):
-                if not (yield ("mbar", lambda i=i: q_full[i].done(0))):
-                    drain_gave_up.add(("Q", i))
-            for kind, ring, issued_n, full in (("K", NK, nk_issued, k_full), ("V", NV, nv_issued, v_full)):
-                for st in range(min(ring, issued_n)):
-                    last = st + ((issued_n - 1 - st) // ring) * ring
-                    if not (yield ("mbar", lambda full=full, st=st, last=last, ring=ring:
-                                   full[st].done((last // ring) & 1))):
-                        drain_gave_up.add((kind, st))
-
-    def named_sync(bar, who, n):
-        g = bar.gen
-        bar.arrive(who, n)
-        return lambda: bar.gen > g
+        if mistake == "no_drain":
+            return
+        # drain: the last load issued into each stage has landed (phase index = tile // ring)
+        for i in range(2):
+            if not (yield ("deadline", lambda i=i: q_full[i].done(0))):
+                drain_gave_up.add(("Q", i))
+        for kind, ring, issued_n, full in (("K", NK, nk_issued, k_full), ("V", NV, nv_issued, v_full)):
+            for st in range(min(ring, issued_n)):
+                last = st + ((issued_n - 1 - st) // ring) * ring
+                if not (yield ("deadline", lambda full=full, st=st, last=last, ring=ring:
+                               full[st].done((last // ring) & 1))):
+                    drain_gave_up.add((kind, st))
 
     def mma():
         q_in = q_full if (fp8 or mistake == "mma_waits_unrotated_q") else q_ready
@@ -232,11 +251,12 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
             issue("S", 1, 0, 0, halves_all)
             commit("s_full", 1)
             commit("k_empty", 0)
-        for j in range(1, nkv + 1):
-            if not ok:
-                break
+        j = 1
+        while ok and j <= nkv:
             jj, sv, sk = j - 1, (j - 1) % NV, j % NK
-            ok = yield ("mbar", lambda sv=sv, jj=jj: v_full[sv].done((jj // NV) & 1))
+            ok = not abort[0]
+            if ok:
+                ok = yield ("mbar", lambda sv=sv, jj=jj: v_full[sv].done((jj // NV) & 1))
             if ok and j < nkv:
                 ok = yield ("mbar", lambda sk=sk, j=j: k_full[sk].done((j // NK) & 1))
             if not ok:
@@ -250,30 +270,36 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
                     issue("PV", i, jj, sv, (0,))
                 yield named_sync(p_ready[i], "mma", 32)
                 issue("PV", i, jj, sv, (1,) if split else halves_all)
-                commit("pv_done", i)
+                if j == nkv:  # the epilogue waits for the last PV only
+                    commit("pv_done", i)
                 commit("v_empty", sv)
                 if j < nkv and not early_s:
                     issue("S", i, j, sk, halves_all)
                 if j < nkv:
                     commit("s_full", i)
                     commit("k_empty", sk)
+                mma_done[i] = j
+            j += 1
+        if not ok and mistake != "mma_leaves_without_schedule":
+            for jd in range(j, nkv + 1):  # the rest of the named-barrier schedule, no MMAs
+                for i in range(2):
+                    if split:
+                        yield named_sync(p_half[i], "mma", 32)
+                    yield named_sync(p_ready[i], "mma", 32)
+                    mma_done[i] = jd
 
     def softmax(i):
         who = f"softmax{i}"
         ok = True
         if not fp8:
-            q_ok = yield ("mbar", lambda: q_full[i].done(0))
-            if q_ok:
+            ok = yield ("mbar", lambda: q_full[i].done(0))
+            if ok:
                 if touching(i, 0):
                     errors.append(f"Q{i} rotated while an MMA reads it")
                 qstate[i] = "rotated"
-            if q_ok or not fixes:
-                q_ready[i].arrive()  # the kernel today arrives whether or not the tile came
-            if fixes:
-                ok = q_ok
-        for j in range(nkv):
-            if not ok:
-                break
+                q_ready[i].arrive()  # only a tile that came is handed on
+        j = 0
+        while ok and j < nkv:
             ok = yield ("mbar", lambda j=j: s_full[i].done(j & 1))
             if not ok:
                 break
@@ -306,8 +332,39 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
                 yield lambda: True
                 if pv_pending(i):
                     errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
+            j += 1
+        if not ok and mistake != "softmax_leaves_without_schedule":
+            # the rest of the named-barrier schedule, no work; each arrival waits until its
+            # partner has passed the previous generation (the pacing the data
+            # dependencies give on the normal path), so arrivals never run a generation
+            # ahead.  Only the MMA warp's progress is published: it passing PReady_1(t-1)
+            # means warpgroup 1 passed Turn_1(t-1) before arriving there, and it passing
+            # PReady_0(t) means warpgroup 0 passed Turn_0(t-1).
+            paced = mistake != "dry_without_pacing"
+            for t in range(j, nkv):
+                turns = pingpong and mistake != "dry_schedule_without_turns"
+                if turns:
+                    if i == 1:
+                        yield named_sync(turn[1], who, 128)
+                    elif t > 0:
+                        yield named_sync(turn[0], who, 128)
+                if paced:
+                    yield lambda t=t: mma_done[i] >= t
+                if split:
+                    p_half[i].arrive(who, 128)
+                if turns:
+                    if i == 0:
+                        if paced:
+                            yield lambda t=t: mma_done[1] >= t
+                        turn[1].arrive(who, 128)
+                    elif t + 1 < nkv:
+                        if paced:
+                            yield lambda t=t: mma_done[0] >= t + 1
+                        turn[0].arrive(who, 128)
+                p_ready[i].arrive(who, 128)
+                yield lambda: True
         if ok:
-            ok = yield ("mbar", lambda: pv_done[i].done((nkv - 1) & 1))
+            ok = yield ("mbar", lambda: pv_done[i].done(0))
         if ok and pv_pending(i):
             errors.append(f"softmax{i} reads O while a PV writes it")
 
@@ -329,15 +386,18 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
             finished.add(name)
 
     hang = []
-    for _ in range(100000):
+    for _ in range(200000):
         if errors and lost is None:
             break
+        if len(finished) == len(roles):
+            break  # every role has ended: the CTA reaches its last barrier
         options = [("role", n) for n in roles if n not in finished and ready(n)]
         options += [("tma", ld) for ld in tma if ld not in stalled]
         if queue:
             options.append(("mma", None))
-        if len(finished) == len(roles):
-            break  # every role has ended: the CTA exits here
+        if abort[0]:  # a waiting role sees the flag and gives up
+            options += [("abort", n) for n in roles if n not in finished and not ready(n)
+                        and isinstance(waiting[n], tuple) and waiting[n][0] == "mbar"]
         if not options:
             blocked = sorted(set(roles) - finished)
             bounded = [n for n in blocked if isinstance(waiting[n], tuple)]
@@ -347,6 +407,8 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
                 break
             name = rng.choice(bounded)
             timeouts.append(name)
+            if waiting[name][0] == "mbar":
+                abort[0] = True
             step(name, False)
             continue
         kind, what = rng.choice(options)
@@ -354,11 +416,23 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, fixes=False, repor
             land(what)
         elif kind == "mma":
             complete_mma()
+        elif kind == "abort":
+            step(what, False)
         else:
             step(what, None if waiting[what] is None else True)
+    else:
+        errors.append("no progress bound reached")
+    # CTA exit: after a failure the MMA thread waits for its own MMAs (they always
+    # complete); on the fault-free path nothing may still be running
+    if abort[0]:
+        while queue:
+            complete_mma()
+    elif lost is None and len(finished) == len(roles) and queue:
+        errors.append(f"{len(queue)} MMAs still running when TMEM is released")
     if report is not None:
         report["in_flight_at_exit"] = list(tma)
         report["drain_gave_up"] = set(drain_gave_up)
+        report["abort"] = abort[0]
     if lost is not None:
         return hang, len(finished) == len(roles), timeouts
     return errors, len(finished) == len(roles), timeouts
@@ -395,81 +469,90 @@ def test_planted_protocol_mistakes_are_caught(mistake, name):
     pytest.fail(f"{mistake} not caught in 400 interleavings")
 
 
-# Faults the bounded waits cover: a K or V load that never lands, a stage release
-# (tcgen05.commit on k_empty / v_empty) that never arrives, and in FP8 (where the
-# MMA warp itself waits for Q) a Q load that never lands.  Every role ends through
-# a wait that times out (the kernel records DIT_ERR_TIMEOUT) and the CTA reaches
-# its exit; none stays blocked on a named barrier.
-COVERED_FAULTS = [("load", "K", 0), ("load", "K", 2), ("load", "K", 5), ("load", "V", 0), ("load", "V", 3),
-                  ("commit", "k_empty", 0, 0), ("commit", "k_empty", 1, 1), ("commit", "v_empty", 0, 0),
-                  ("commit", "v_empty", 1, 1)]
+def _faults(cfg):
+    """Every single loss the model can inject for a 7-tile run: each TMA load (Q, K,
+    V), each stage release and each S / PV completion signal."""
+    out = [("load", "Q", 0), ("load", "Q", 1)]
+    out += [("load", kind, t) for kind in ("K", "V") for t in range(7)]
+    out += [("commit", "pv_done", 0, 0), ("commit", "pv_done", 1, 0)]
+    for name, n, per in (("k_empty", cfg["NK"], 2), ("v_empty", cfg["NV"], 2), ("s_full", 2, 1)):
+        for idx in range(n):
+            uses = 7 if name == "s_full" else -(-7 // n) * per
+            out += [("commit", name, idx, k) for k in sorted({0, uses // 2, uses - 2, uses - 1})]
+    return out
+
+
+def _waited_on(fault, cfg, nkv):
+    """Whether some wait depends on the lost arrival: every load, S completion and
+    the (single) completion of the last PV; the stage release of tile t only if
+    tile t + ring is loaded into that stage."""
+    if fault[0] == "load" or fault[1] in ("s_full", "pv_done"):
+        return True
+    _, name, idx, n = fault
+    ring = cfg["NK"] if name == "k_empty" else cfg["NV"]
+    return idx + (n // 2) * ring + ring < nkv
 
 
 @pytest.mark.parametrize("name", sorted(CONFIGS))
-@pytest.mark.parametrize("fault", COVERED_FAULTS, ids=lambda f: "-".join(map(str, f)))
-def test_lost_loads_and_releases_end_every_role(name, fault):
-    for seed in range(100):
-        hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=fault, **CONFIGS[name])
-        assert finished and not hang, (name, fault, seed, hang)
-        assert timeouts, (name, fault, seed)  # the loss is reported, not absorbed
-
-
-def test_lost_q_load_ends_every_role_in_fp8():
-    for seed in range(100):
-        hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=("load", "Q", 0), **CONFIGS["fp8_d128"])
-        assert finished and not hang and timeouts, (seed, hang)
-
-
-# Faults the bounded waits do not cover (named barriers cannot time out), found
-# by this model.  Both need a lost hardware arrival; the fault-free protocol
-# above never produces one.
-#  * s_full: if the tensor core's arrival is lost, the softmax warpgroup times out
-#    and leaves its loop without arriving at its P-ready named barrier, where the
-#    MMA warp then waits without a limit.
-#  * BF16 Q load: the softmax warpgroup that rotates Q arrives on q_ready even when
-#    its wait for the tile timed out, so the MMA warp may go on into the named
-#    barriers while the other warpgroup's wait times out (which timeout fires
-#    first decides).  Arriving on q_ready only when the tile came would close it.
-UNCOVERED_FAULTS = [(n, ("commit", "s_full", 0, 1)) for n in sorted(CONFIGS)] + \
-                   [(n, ("load", "Q", 0)) for n in ("bf16_d128", "bf16_d64")]
-
-
-@pytest.mark.parametrize("name,fault", UNCOVERED_FAULTS, ids=lambda x: x if isinstance(x, str) else "-".join(map(str, x)))
-def test_uncovered_faults_end_at_a_named_barrier(name, fault):
-    for seed in range(100):
-        hang, finished, _ = simulate(nkv=7, seed=seed, lost=fault, **CONFIGS[name])
-        if hang:
-            assert "mma" in hang[0] and "named barriers" in hang[0], hang
-            return
-    pytest.fail(f"{fault} ended every role in 100 interleavings")
+def test_every_single_loss_ends_every_role(name):
+    """Whatever arrival is lost, every role ends (the loss is reported through a
+    bounded wait that gives up, never absorbed silently into a hang), and a load
+    still in flight when the CTA ends is one the producer's drain waited for."""
+    cfg = CONFIGS[name]
+    faults = _faults(cfg)
+    assert len(faults) > 30
+    for fault in faults:
+        for seed in range(40):
+            rep = {}
+            hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=fault, report=rep, **cfg)
+            assert finished and not hang, (name, fault, seed, hang)
+            for kind, slot, _ in rep["in_flight_at_exit"]:
+                assert (kind, slot) in rep["drain_gave_up"], (fault, seed, rep)
+            if _waited_on(fault, cfg, 7):
+                assert timeouts and rep["abort"], (name, fault, seed)
+            else:  # nothing waits for it: the loss changes nothing
+                assert not timeouts and not rep["abort"], (name, fault, seed)
 
 
 @pytest.mark.parametrize("name", sorted(CONFIGS))
-def test_planned_failure_path_fixes(name):
-    """The planned changes, checked on the model before they go into the kernel:
-    fault-free runs stay free of hazards and of timeouts (so the drain's parity
-    formula is right) and end with nothing in flight; every load loss, Q included,
-    now ends every role; and a load still in flight when the roles end is always
-    one the drain waited for and gave up on."""
+def test_fault_free_runs_raise_no_abort_and_leave_nothing_in_flight(name):
     cfg = CONFIGS[name]
     for nkv in (1, 2, 3, 5, 9):
         for seed in range(150):
             rep = {}
-            errors, finished, timeouts = simulate(nkv=nkv, seed=seed, fixes=True, report=rep, **cfg)
-            assert not errors and finished and not timeouts and not rep["in_flight_at_exit"], (nkv, seed, errors)
-    for fault in COVERED_FAULTS + [("load", "Q", 0), ("load", "Q", 1)]:
-        for seed in range(100):
-            rep = {}
-            hang, finished, timeouts = simulate(nkv=7, seed=seed, lost=fault, fixes=True, report=rep, **cfg)
-            assert finished and not hang and timeouts, (fault, seed, hang)
-            for kind, slot, _ in rep["in_flight_at_exit"]:
-                assert (kind, slot) in rep["drain_gave_up"], (fault, seed, rep)
+            errors, finished, timeouts = simulate(nkv=nkv, seed=seed, report=rep, **cfg)
+            assert not errors and finished and not timeouts, (nkv, seed, errors)
+            assert not rep["in_flight_at_exit"] and not rep["abort"], (nkv, seed, rep)
 
 
-def test_without_the_drain_a_stalled_load_is_left_behind_unwaited():
-    """Today's kernel: after a load stalls, the CTA ends with it in flight and no
-    wait for it (the planned drain waits for it, bounded, before leaving)."""
+# Planted mistakes in the failure path: each leaves some role on a named barrier
+# (or exits with a load in flight) under some single loss.
+FAILURE_PATH_MISTAKES = [
+    ("dry_without_pacing", "bf16_d128", ("load", "Q", 0)),
+    ("dry_without_pacing", "fp8_d128", ("load", "V", 2)),
+    ("softmax_leaves_on_timeout", "fp8_d128", ("commit", "s_full", 0, 2)),
+    ("softmax_leaves_on_timeout", "bf16_d128", ("commit", "s_full", 1, 2)),
+    ("dry_schedule_without_turns", "bf16_d128", ("commit", "s_full", 0, 2)),
+    ("mma_leaves_without_schedule", "bf16_d64", ("load", "V", 3)),
+]
+
+
+@pytest.mark.parametrize("mistake,name,fault", FAILURE_PATH_MISTAKES)
+def test_planted_failure_path_mistakes_hang(mistake, name, fault):
+    m = {"softmax_leaves_on_timeout": "softmax_leaves_without_schedule"}.get(mistake, mistake)
+    for seed in range(200):
+        hang, finished, _ = simulate(nkv=7, seed=seed, lost=fault, mistake=m, **CONFIGS[name])
+        if hang or not finished:
+            return
+    pytest.fail(f"{mistake} under {fault} never hung in 200 interleavings")
+
+
+def test_without_the_drain_a_stalled_load_is_left_behind():
     rep = {}
-    hang, finished, _ = simulate(nkv=7, seed=0, lost=("load", "K", 2), report=rep, **CONFIGS["bf16_d128"])
-    assert finished and not hang
-    assert ("K", 2 % 3, 2) in rep["in_flight_at_exit"] and not rep["drain_gave_up"]
+    for seed in range(50):
+        hang, finished, _ = simulate(nkv=7, seed=seed, lost=("load", "K", 2), mistake="no_drain", report=rep,
+                                     **CONFIGS["bf16_d128"])
+        assert finished and not hang
+        if ("K", 2 % 3, 2) in rep["in_flight_at_exit"] and not rep["drain_gave_up"]:
+            return
+    pytest.fail("a stalled load was never left in flight without the drain")

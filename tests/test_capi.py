@@ -1,9 +1,11 @@
 """C-ABI checks that need no GPU: the library loads, exports every symbol that
 include/dit.h declares, and rejects bad arguments before touching a device."""
 import ctypes
+import math
 import os
 import re
 
+import numpy as np
 import pytest
 
 from diffusion_transformer_denoising_dit_b200 import _binding as B
@@ -95,6 +97,38 @@ def test_small_outputs_alignment():
     assert L.fbcache_gate_noalloc(A16, A16, 100, 0.1, A16 + 2, A16, None) == 3
     assert L.fbcache_gate_finalize(A16, 0.1, A16, A16 + 2, None) == 3
     assert L.dit_rope_tables(A16 + 2, 10, 16, 24, 24, 1e4, A16, A16, None) == 3        # pos
+
+
+def test_gate_reference_update_argument_checks():
+    L = B.lib()
+    assert L.fbcache_gate_ref_update(None, A16, 64, None, None) == 1          # null input
+    assert L.fbcache_gate_ref_update(A16, A16, 64, None, None) == 1           # r_ref == r_cur
+    assert L.fbcache_gate_ref_update(A16, A16 + 4096, 0, None, None) == 1     # n < 1
+    assert L.fbcache_gate_ref_update(A16 + 2, A16 + 4096, 64, None, None) == 3
+    assert L.fbcache_gate_ref_update(A16, A16 + 4096, 64, A16 + 2, None) == 3  # misaligned flag
+
+
+def test_integer_qk_variant_shares_the_fp8_argument_checks():
+    L = B.lib()
+    st = S(1 << 20, 1 << 20, 128)
+    args = (A16, A16, A16, A16 + (1 << 24), 1, 1, 1024, 128, st, st, st, st, None, None, 0.0)
+    assert L.dit_attn_fp8_i8qk(*args, 64, 64, 1, A16, 1 << 30, None) == 2     # q_block != 128
+    assert L.dit_attn_fp8_i8qk(*args, 128, 64, 1, None, 0, None) == 4         # no workspace
+    args64 = (A16, A16, A16, A16 + (1 << 24), 1, 1, 1024, 64, st, st, st, st, None, None, 0.0)
+    assert L.dit_attn_fp8_i8qk(*args64, 128, 64, 1, A16, 1 << 30, None) == 2  # d = 64
+
+
+def test_gate_entry_points_agree_on_thresholds():
+    """fbcache_gate and fbcache_gate_noalloc accept and refuse the same thresholds:
+    NaN and +-inf are refused, every finite float (FLT_MAX included) passes the
+    argument checks (and then meets the device check, with no GPU here)."""
+    L = B.lib()
+    flt_max = float(np.finfo(np.float32).max)
+    for thr in (float("nan"), float("inf"), -float("inf"), flt_max, -flt_max, 3.4e38, 0.0, 0.12):
+        a = L.fbcache_gate(A16, A16, 100, thr, A16, A16, A16, 1 << 20, None)
+        b = L.fbcache_gate_noalloc(A16, A16, 100, thr, A16, A16, None)
+        assert a == b, (thr, a, b)
+        assert a == (1 if not math.isfinite(thr) else 2), (thr, a)
 
 
 def test_skippable_attention_argument_validation():

@@ -182,6 +182,38 @@ def test_gate_last_computed_policy_matches_oracle():
     assert dit.read_error() == 0
 
 
+@pytest.mark.parametrize("policy", ["consecutive", "last_computed"])
+@pytest.mark.parametrize("warmup", [1, 4])
+def test_gate_policies_on_the_device_match_oracle(policy, warmup):
+    """FBCacheGate.step over the 28-step drift with the reference residual kept on
+    the device (no host read inside the loop): the per-step flags equal the
+    oracle's decisions under both policies and warm-up lengths."""
+    res = [r.to(DEV) for r in synth.drift_residuals(1024, 512, steps=28)]
+    ref = G.trace_decisions([r.cpu() for r in res], 0.12, policy=policy, warmup=warmup)
+    gate = dit.FBCacheGate(0.12, res[0].numel(), device=DEV, policy=policy, warmup=warmup)
+    flags = torch.full((28,), -1, dtype=torch.int32, device=DEV)
+    for t in range(28):
+        flags[t:t + 1].copy_(gate.step(res[t]))
+    got = [bool(x) for x in flags.tolist()]
+    assert got == [s for _, s in ref], (got, [s for _, s in ref])
+    assert dit.read_error() == 0
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 2049, 1000003])
+def test_gate_reference_update_follows_the_flag(n):
+    """fbcache_gate_ref_update copies r_cur into r_ref exactly when the flag is 0
+    (and always without a flag), ragged sizes included."""
+    g = torch.Generator(device=DEV).manual_seed(n)
+    cur = torch.randn(n, generator=g, device=DEV).to(torch.bfloat16)
+    for flag_val, want_copy in ((None, True), (0, True), (1, False)):
+        ref = torch.full((n,), 7.0, device=DEV, dtype=torch.bfloat16)
+        flag = None if flag_val is None else torch.full((1,), flag_val, dtype=torch.int32, device=DEV)
+        dit.fbcache_gate_ref_update(cur, ref, flag)
+        torch.cuda.synchronize()
+        assert torch.equal(ref, cur) if want_copy else bool((ref == 7.0).all()), (flag_val, n)
+    assert dit.read_error() == 0
+
+
 def test_gate_sums_and_finalize_reproduce_the_gate():
     """fbcache_gate_sums + fbcache_gate_finalize on the whole tensor give fbcache_gate's
     rel bit for bit; from two shards' totals added together, the same decision."""

@@ -58,8 +58,10 @@ def test_every_source_compiles_its_kernels(reports):
 
 # Known spills, per kernel: (store bytes, load bytes) allowed.  kmean_partial (the
 # K-mean pass of the FP8 prologue, 33 us of a 2.7 ms FP8 call) keeps one 4-byte
-# value on the stack at 40 registers.
-SPILL_ALLOWANCE = {"kmean_partial": (4, 12)}
+# value on the stack at 40 registers.  The quantiser's int8 instantiation
+# (quantize_qkv<true>) holds its 64 tile values in registers at the 80-register
+# cap of three CTAs per SM and keeps four words of the int8 packing on the stack.
+SPILL_ALLOWANCE = {"kmean_partial": (4, 12), "quantize_qkvILb1E": (16, 24)}
 
 
 def test_no_register_spills(reports):
@@ -91,4 +93,4 @@ def test_register_resplit_fits_the_launch_registers(reports):
                 continue
             found += 1
             assert need <= threads * regs, (name, regs, need, threads * regs)
-    assert found == 3  # <bf16, 64>, <bf16, 128>, <fp8, 128>
+    assert found == 4  # <bf16, 64>, <bf16, 128>, <fp8, 128>, <fp8, 128, integer Q.K^T>

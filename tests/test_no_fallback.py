@@ -48,12 +48,14 @@ def test_entry_points_report_unsupported_without_an_sm100_device():
     args8 = (A16, A16, A16, O, 1, 1, 16, 128, st8, st8, st8, st8, None, None, 0.0)
     need = L.dit_attn_fp8_workspace_bytes(1, 1, 16, 128, 128, 64)
     assert L.dit_attn_fp8(*args8, 128, 64, 1, A16, need, None) == DIT_ERR_UNSUPPORTED
+    assert L.dit_attn_fp8_i8qk(*args8, 128, 64, 1, A16, need, None) == DIT_ERR_UNSUPPORTED
     assert L.rope_apply(A16, A16, 1, 1, 16, 64, st, st, A16, A16, 0, None) == DIT_ERR_UNSUPPORTED
     assert L.dit_rope_tables(A16, 16, 16, 24, 24, 1e4, A16, A16, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate(A16, A16, 64, 0.1, A16, A16, A16, 1 << 20, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate_noalloc(A16, A16, 64, 0.1, A16, A16, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate_sums(A16, A16, 64, A16, A16, 1 << 20, None) == DIT_ERR_UNSUPPORTED
     assert L.fbcache_gate_finalize(A16, 0.1, A16, A16, None) == DIT_ERR_UNSUPPORTED
+    assert L.fbcache_gate_ref_update(A16, A16 + 4096, 64, None, None) == DIT_ERR_UNSUPPORTED
     assert L.dit_selftest_wait_timeout(None) == DIT_ERR_UNSUPPORTED
     assert L.dit_read_error(None) == DIT_ERR_UNSUPPORTED
 
