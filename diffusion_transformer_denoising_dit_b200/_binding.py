@@ -13,10 +13,11 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdit.so")
+# DIT_LIB_VARIANT=debug loads the bounds-checking debug build (libdit_debug.so)
+LIB_PATH = os.path.join(_PKG, "libdit_debug.so" if os.environ.get("DIT_LIB_VARIANT") == "debug" else "libdit.so")
 
 STATUS = {0: "DIT_OK", 1: "DIT_ERR_INVALID_ARG", 2: "DIT_ERR_UNSUPPORTED", 3: "DIT_ERR_ALIGNMENT",
-          4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT"}
+          4: "DIT_ERR_WORKSPACE", 5: "DIT_ERR_LAUNCH", 6: "DIT_ERR_TIMEOUT", 7: "DIT_ERR_BOUNDS"}
 EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply",
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
            "dit_attn_fp8", "dit_attn_fp8_i8qk", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",

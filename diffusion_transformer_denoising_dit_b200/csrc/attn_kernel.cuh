@@ -162,7 +162,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 // Out of line, so that its registers stay out of the softmax branch's allocation.
 template <int D, typename Wait>
 __device__ __noinline__ bool rotate_q_tile(uint8_t* q_tile, const float* rope_cos, const float* rope_sin, int qrow0,
-                                           int N, Wait wait_tile) {
+                                           int N, Wait wait_tile, int* err) {
   constexpr int kSubBytes = 128 * 128;  // one 128-row, 128-byte column block
   constexpr int CPR = D / 8;            // 16-byte chunks per row
   constexpr int RPP = 128 / CPR;        // rows covered per pass
@@ -188,7 +188,9 @@ __device__ __noinline__ bool rotate_q_tile(uint8_t* q_tile, const float* rope_co
   for (int k = 0; k < NP; ++k) {
     // row r's chunk c sits at column block c / 8, 16-byte slot (c % 8) ^ (r % 8) (128-byte swizzle)
     const int r = r0 + RPP * k;
-    uint4* p = reinterpret_cast<uint4*>(q_tile + r * 128 + (c >> 3) * kSubBytes + (((c & 7) ^ (r & 7)) << 4));
+    const int off = r * 128 + (c >> 3) * kSubBytes + (((c & 7) ^ (r & 7)) << 4);
+    if (!debug_check(off >= 0 && off + 16 <= 128 * D * 2, err)) continue;  // within the bf16 Q tile
+    uint4* p = reinterpret_cast<uint4*>(q_tile + off);
     const uint4 xv = *p;
     const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
     const float cc[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w}, ss[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
@@ -307,8 +309,10 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(q_full + i, C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sQ + i * C::kTileBytes + c * C::kSubBytes, &tmQ, q_full + i, c * C::kBoxInner,
-                      (2 * qt + i) * BM, h, b);
+          if (debug_check((c * C::kBoxInner * C::EB) % 16 == 0 && i * C::kTileBytes + (c + 1) * C::kSubBytes <=
+                              2 * C::kTileBytes, err))  // 16-byte x coordinate; inside the Q tiles
+            tma_load_4d(sQ + i * C::kTileBytes + c * C::kSubBytes, &tmQ, q_full + i, c * C::kBoxInner,
+                        (2 * qt + i) * BM, h, b);
       }
       int nk_issued = 0, nv_issued = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -317,13 +321,17 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(k_full + sk, C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sK + sk * C::kTileBytes + c * C::kSubBytes, &tmK, k_full + sk, c * C::kBoxInner, j * BN, h, b);
+          if (debug_check(sk < NK && j * BN < N && (c * C::kBoxInner * C::EB) % 16 == 0, err))
+            tma_load_4d(sK + sk * C::kTileBytes + c * C::kSubBytes, &tmK, k_full + sk, c * C::kBoxInner, j * BN, h,
+                        b);
         ++nk_issued;
         if (j >= NV && !mbar_wait(v_empty + sv, ((j / NV) & 1) ^ 1, err, kErrTimeout, abort_flag)) break;
         mbar_arrive_expect_tx(v_full + sv, C::kTileBytes);
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sV + sv * C::kTileBytes + c * C::kSubBytes, &tmV, v_full + sv, c * C::kBoxInner, j * BN, h, b);
+          if (debug_check(sv < NV && j * BN < N && (c * C::kBoxInner * C::EB) % 16 == 0, err))
+            tma_load_4d(sV + sv * C::kTileBytes + c * C::kSubBytes, &tmV, v_full + sv, c * C::kBoxInner, j * BN, h,
+                        b);
         ++nv_issued;
       }
       // Drain: the last load issued into every stage has landed before the CTA
@@ -351,6 +359,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t v_addr = smem_u32(sV);
       auto qk = [&](int i, int sk) {  // S_i = Q_i K^T
         const uint32_t qa = q_addr + i * C::kTileBytes, ka = k_addr + sk * C::kTileBytes;
+        // S_i's columns end before O's; the K stage is one of the ring's
+        if (!debug_check(i < 2 && sk < NK && C::kColS + 128 * i + BN <= C::kColO, err)) return;
 #pragma unroll
         for (int kk = 0; kk < D / C::kKStep; ++kk) {
           const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;  // 32 bytes of K per MMA
@@ -367,6 +377,10 @@ __global__ void __launch_bounds__(384, 1)
       // overwrites O_i when acc is false (first tile)
       auto pv = [&](int i, int sv, bool acc, int k0, int k1) {
         const uint32_t va = v_addr + sv * C::kTileBytes;
+        // O_i inside the allocation, P inside S_i, the V stage one of the ring's
+        if (!debug_check(i < 2 && sv < NV && C::kColO + D * (i + 1) <= C::kTmemCols && k1 * 8 <= BN &&
+                             k0 >= 0, err))
+          return;
 #pragma unroll
         for (int kk = k0; kk < k1; ++kk) {
           // kKStep keys = kKStep rows of 128 bytes; d column blocks are kSubBytes apart
@@ -477,8 +491,8 @@ __global__ void __launch_bounds__(384, 1)
     if constexpr (!FP8) {
       uint64_t* qf = q_full + i;
       auto wait_tile = [qf, err, abort_flag]() { return mbar_wait(qf, 0, err, kErrTimeout, abort_flag); };
-      ok = __all_sync(0xffffffffu,
-                      rotate_q_tile<D>(sQ + i * C::kTileBytes, out.rope_cos, out.rope_sin, qblk * BM, N, wait_tile));
+      ok = __all_sync(0xffffffffu, rotate_q_tile<D>(sQ + i * C::kTileBytes, out.rope_cos, out.rope_sin, qblk * BM, N,
+                                                    wait_tile, err));
       // the MMA reads Q through the async proxy: order the generic-proxy writes first
       fence_proxy_async_smem();
       // only a tile that came is handed on; otherwise the MMA warp's bounded wait gives up
@@ -488,6 +502,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + C::kColS + 128 * i + lane_off;
     const uint32_t tO = tmem + C::kColO + D * i + lane_off;
+    // this warp's lanes and the S_i / O_i columns inside the 512-column allocation
+    debug_check((warp & 3) * 32 + 32 <= 128 && C::kColS + 128 * i + BN <= C::kColO &&
+                    C::kColO + D * (i + 1) <= C::kTmemCols, err);
     const float sl2 = out.scale_log2;
     // FP8 scales: score = S * sQ * sK(j) * scale, P8 = p * 2^-tau * 448 * sV(j) / sV_max
     float qs = sl2, vfold = 1.f, fin_scale = 1.f;

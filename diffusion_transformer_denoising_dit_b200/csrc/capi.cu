@@ -116,6 +116,7 @@ const char* dit_status_string(dit_status s) {
     case DIT_ERR_WORKSPACE: return "DIT_ERR_WORKSPACE";
     case DIT_ERR_LAUNCH: return "DIT_ERR_LAUNCH";
     case DIT_ERR_TIMEOUT: return "DIT_ERR_TIMEOUT";
+    case DIT_ERR_BOUNDS: return "DIT_ERR_BOUNDS";
   }
   return "DIT_ERR_UNKNOWN";
 }

@@ -35,6 +35,18 @@ __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Bounds checks of the debug build (compiled with -DDIT_DEBUG): a failed check
+// records kErrBounds in the error word and the caller skips the access; no trap.
+// In the normal build the check is the constant true and compiles away.
+#ifdef DIT_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok, int* err) {
+  if (!ok) set_error(err, kErrBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool debug_check(bool, int*) { return true; }
+#endif
+
 // ----------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------

@@ -13,6 +13,7 @@ constexpr int kAttnBlockN = 128;
 
 // Error codes written to the device error word (match dit_status).
 constexpr int kErrTimeout = 6;
+constexpr int kErrBounds = 7;  // debug builds only (DIT_DEBUG): an index failed its bounds check
 
 // Gate: number of pass-1 CTAs for n elements, and its workspace (2 doubles per CTA).
 int gate_num_ctas(int64_t n);

@@ -80,7 +80,9 @@ typedef enum {
   DIT_ERR_ALIGNMENT = 3,    /* pointer or stride not 16-byte aligned */
   DIT_ERR_WORKSPACE = 4,    /* workspace missing or too small */
   DIT_ERR_LAUNCH = 5,       /* CUDA error while enqueueing */
-  DIT_ERR_TIMEOUT = 6       /* (device error word) a bounded wait ran out */
+  DIT_ERR_TIMEOUT = 6,      /* (device error word) a bounded wait ran out */
+  DIT_ERR_BOUNDS = 7        /* (device error word, debug build libdit_debug.so only) an index
+                               failed a device-side bounds check; the access was skipped */
 } dit_status;
 
 /* Human-readable name of a status code (static string). */

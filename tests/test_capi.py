@@ -25,6 +25,15 @@ def test_header_declares_the_binding_exports():
     assert _declared() == sorted(B.EXPORTS)
 
 
+def test_debug_build_exports_every_declared_symbol():
+    path = os.path.join(os.path.dirname(B.LIB_PATH), "libdit_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libdit_debug.so not built (run build())")
+    L = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
 def test_library_exports_every_declared_symbol():
     L = B.lib()
     for name in _declared():
