@@ -698,6 +698,30 @@ def run_fp8_peak():
                       "clocks": clk.summary()}), flush=True)
 
 
+def run_profile_case(args):
+    """A short, fixed invocation for ncu captures: `calls` attention calls of one
+    precision on one workload (inputs and workspace allocated once, about 1 GB on
+    the device for the 2048-px workload), then the cache gate once."""
+    import torch
+    import diffusion_transformer_denoising_dit_b200 as dit
+    from diffusion_transformer_denoising_dit_b200 import synth
+    dev = torch.device("cuda", 0)
+    w = synth.WORKLOADS[args.profile_workload]
+    q, k, v = synth.qkv(w, device=dev)
+    pos = synth.positions(w.T, w.G).to(dev)
+    cos, sin = dit.rope_tables(pos, w.axes, w.theta)
+    o = torch.empty_like(q)
+    prec = args.profile_attn
+    ws = dit.attention_workspace(w.B, w.H, w.N, w.d, "bf16" if prec == "bf16" else "fp8", device=dev)
+    for _ in range(args.profile_calls):
+        dit.attention(q, k, v, cos, sin, precision=prec, out=o, workspace=ws)
+    r_prev, r_cur = synth.gate_pair(w.N, HIDDEN, 0.05, device=dev)
+    dit.fbcache_gate(r_cur.contiguous(), r_prev.contiguous(), THRESHOLD)
+    torch.cuda.synchronize()
+    assert dit.read_error() == 0
+    print(json.dumps({"profile_case": prec, "workload": w.name, "calls": args.profile_calls}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -708,6 +732,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--trace", action="store_true", help="run the 28-step denoising trace instead")
     ap.add_argument("--measure-fp8-peak", action="store_true", help="dense e4m3 GEMM peak (a denominator) instead")
+    ap.add_argument("--profile-attn", choices=["bf16", "fp8", "fp8_i8qk"],
+                    help="a short fixed invocation for ncu captures instead of the benchmark")
+    ap.add_argument("--profile-workload", default=WORKLOAD, choices=["flux1k", "flux2k"])
+    ap.add_argument("--profile-calls", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -722,6 +750,9 @@ def main():
         return
     if args.measure_fp8_peak:
         run_fp8_peak()
+        return
+    if args.profile_attn:
+        run_profile_case(args)
         return
     if world > 1:
         import datetime

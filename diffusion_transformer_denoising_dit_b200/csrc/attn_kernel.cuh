@@ -211,6 +211,26 @@ __device__ __noinline__ bool rotate_q_tile(uint8_t* q_tile, const float* rope_co
   return true;
 }
 
+// Named barriers of the attention kernel (0 is __syncthreads): P-ready of
+// softmax warpgroup i (128 arrivals + the MMA warp's 32), the ping-pong turns
+// (256), and BF16's first-half P hand-off (160).
+constexpr uint32_t kBarPReady = 1, kBarTurn = 3, kBarPHalf = 5;
+
+// The MMA warp's failure path: the rest of its named-barrier schedule from
+// iteration j (every P-half and P-ready sync it would have made, without the
+// MMAs), publishing its progress after each P-ready as the normal path does.
+template <bool kSplitP>
+__device__ __noinline__ void mma_warp_finish_schedule(int j, int nkv, uint32_t mma_done, bool leader) {
+  for (; j <= nkv; ++j) {
+    if constexpr (kSplitP) named_sync<kBarPHalf + 0, 160>();
+    named_sync<kBarPReady + 0, 160>();
+    if (leader) flag_store(mma_done, j);
+    if constexpr (kSplitP) named_sync<kBarPHalf + 1, 160>();
+    named_sync<kBarPReady + 1, 160>();
+    if (leader) flag_store(mma_done + 4, j);
+  }
+}
+
 // I8QK (FP8 only): Q and K are symmetric int8 and S = Q K^T is a kind::i8 MMA
 // with s32 accumulation (exact: |S| <= 127^2 * 128 < 2^22); P.V stays e4m3.
 template <bool FP8, int D, bool I8QK = false>
@@ -240,7 +260,6 @@ __global__ void __launch_bounds__(384, 1)
   // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
   //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
   //                 kBarPHalf + i   BF16: softmax i stored keys 0..63 of P (128 arrive, MMA warp syncs)
-  constexpr uint32_t kBarPReady = 1, kBarTurn = 3, kBarPHalf = 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
   // Raised by the first role whose bounded wait gives up; every other bounded
   // wait then gives up too.  A role that gives up still performs the rest of its
@@ -466,17 +485,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         __syncwarp();
       }
-      if (!ok) {
-        // Failure path: the rest of the named-barrier schedule, no MMAs.
-        for (; j <= nkv; ++j) {
-          if constexpr (C::kSplitP) named_sync<kBarPHalf + 0, 160>();
-          named_sync<kBarPReady + 0, 160>();
-          if (leader) flag_store(mma_done, j);
-          if constexpr (C::kSplitP) named_sync<kBarPHalf + 1, 160>();
-          named_sync<kBarPReady + 1, 160>();
-          if (leader) flag_store(mma_done + 4, j);
-        }
-      }
+      // Failure path: the rest of the named-barrier schedule, no MMAs (out of line:
+      // inline, its loop cost the normal path 6 % of the cycles in BF16, measured)
+      if (!ok) mma_warp_finish_schedule<C::kSplitP>(j, nkv, mma_done, leader);
    }
   } else {
     regs_inc<C::kRegsSoftmax>();

@@ -64,6 +64,60 @@ def attention(q, k, v, cos=None, sin=None, group=None, attend=None, **kwargs):
     return head_to_seq(attend(qh, kh, vh, cos, sin, **kwargs), group)
 
 
+def _seq_to_head_chunk(x, c, chunks, group):
+    """Start the exchange of head chunk c: every rank sends rank r its tokens of
+    rank r's chunk-c heads ([B, H / P / chunks, n, d] per destination).  Returns
+    the receive buffer [P, B, H / P / chunks, n, d] and the async work."""
+    P = dist.get_world_size(group)
+    B, H, n, d = x.shape
+    Hp = H // P
+    Hc = Hp // chunks
+    send = x.reshape(B, P, chunks, Hc, n, d)[:, :, c].permute(1, 0, 2, 3, 4).contiguous()
+    recv = torch.empty_like(send)
+    work = dist.all_to_all_single(recv, send, group=group, async_op=True)
+    return recv, work
+
+
+def _head_chunk_of(recv):
+    """[P, B, Hc, n, d] received blocks -> [B, Hc, P n, d] (all tokens of the chunk's heads)."""
+    P, B, Hc, n, d = recv.shape
+    return recv.permute(1, 2, 0, 3, 4).reshape(B, Hc, P * n, d)
+
+
+def attention_overlapped(q, k, v, cos=None, sin=None, group=None, attend=None, chunks=2, **kwargs):
+    """ulysses.attention with the exchanges split by head chunk and overlapped
+    with the attention of the neighbouring chunks: chunk c + 1's Q, K, V are in
+    flight while chunk c's attention runs, and chunk c's output goes back while
+    chunk c + 1's runs.  chunks must divide H / P; chunks = 1 is the plain form.
+    The result is the same as ulysses.attention's, bit for bit (the same local
+    attention on the same heads).  On NCCL the exchanges run on the collective
+    stream and each wait orders only the launching stream, never the host."""
+    attend = _binding.attention if attend is None else attend
+    P = dist.get_world_size(group)
+    B, H, n, d = q.shape
+    if H % P or (H // P) % chunks:
+        raise ValueError(f"{H} heads do not split over {P} ranks x {chunks} chunks")
+    Hp, Hc = H // P, H // P // chunks
+    inflight = [_seq_to_head_chunk(t, 0, chunks, group) for t in (q, k, v)]
+    outs = []
+    for c in range(chunks):
+        for _, work in inflight:
+            work.wait()
+        qh, kh, vh = (_head_chunk_of(recv) for recv, _ in inflight)
+        if c + 1 < chunks:  # the next chunk's exchange overlaps this chunk's attention
+            inflight = [_seq_to_head_chunk(t, c + 1, chunks, group) for t in (q, k, v)]
+        o = attend(qh, kh, vh, cos, sin, **kwargs)          # [B, Hc, P n, d]
+        send = o.reshape(B, Hc, P, n, d).permute(2, 0, 1, 3, 4).contiguous()  # block r: rank r's tokens
+        recv = torch.empty_like(send)
+        outs.append((recv, dist.all_to_all_single(recv, send, group=group, async_op=True)))
+    res = torch.empty(P, chunks, B, Hc, n, d, dtype=outs[0][0].dtype, device=outs[0][0].device)
+    for c, (recv, work) in enumerate(outs):
+        work.wait()
+        res[:, c] = recv                                      # [P, B, Hc, n, d] from rank s: its heads
+    # heads of rank s, chunk c, index i -> global head s Hp + c Hc + i
+    return res.permute(2, 0, 1, 3, 4, 5).reshape(B, H, n, d)
+
+
 def gate(r_cur, r_prev, threshold: float, group=None, sums=None, finalize=None):
     """First-Block-Cache decision over a residual split across ranks: each rank
     passes its shard; all ranks return the same (rel, skip).

@@ -41,6 +41,8 @@ def test_one_rank_ulysses_equals_the_plain_call(group):
     ref = dit.attention(q, k, v, cos, sin)
     got = ulysses.attention(q, k, v, cos, sin)
     assert torch.equal(got, ref)
+    for chunks in (2, 4):  # head chunks overlapped with the exchanges: the same kernels per head
+        assert torch.equal(ulysses.attention_overlapped(q, k, v, cos, sin, chunks=chunks), ref)
     cur, prev = synth.gate_pair(4608, 768, 0.05, device="cuda")
     rel, skip = ulysses.gate(cur, prev, 0.12)
     rel_ref, skip_ref = dit.fbcache_gate(cur, prev, 0.12)

@@ -82,6 +82,10 @@ def _ulysses_worker(rank, world, port, q):
         o = ulysses.attention(qs.double(), ks.double(), vs.double(), attend=attend)
         full = A.attention(qf, kf, vf, pos=pos.numpy(), axes=w.axes, theta=w.theta)
         err = float(np.abs(o.numpy() - full[:, :, sl]).max())
+        # the overlapped form, head chunk by head chunk: the same result bit for bit
+        for chunks in [c for c in (1, 2, 4) if (w.H // world) % c == 0]:
+            oo = ulysses.attention_overlapped(qs.double(), ks.double(), vs.double(), attend=attend, chunks=chunks)
+            err = max(err, float((oo - o).abs().max()) * 1e12)
         # sharded gate: shard totals, all-reduce, one decision everywhere
         cur, prev = synth.gate_pair(288, 128, 0.1)
         m = 288 // world
