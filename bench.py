@@ -52,6 +52,12 @@ FP8_GEMM_SUSTAINED_RECORDED = 2594.0
 # These are capture results, not measurements of this run; a kernel whose source
 # changed since its capture reports null.
 NCU_TRAFFIC = {
+    # attn_kernel<bf16, d=128>, 2048-px workload: 322.1 MB read + 86.2 MB written
+    ("attn_bf16", "21b926a88b5d1397"): 408_256_256,
+    # attn_kernel<fp8, d=128> (one hash covers both Q.K^T forms' source):
+    # e4m3 Q.K^T 156.0 + 71.5 MB; integer Q.K^T 155.9 + 69.8 MB
+    ("attn_fp8", "db72042d2fd5c9f8"): 227_439_616,
+    ("attn_fp8_i8qk", "db72042d2fd5c9f8"): 225_738_752,
 }
 
 
@@ -396,6 +402,11 @@ def run_ours(args, rank, world, local_rank):
             "peak_nominal_ratio": fp8_peak, "frac_of_step_vs_2x_bf16": v8 / 1e12 / fp8_peak,
             "clocks": c8, "sm_mcycles_per_step": mcycles(mps8, c8),
             "step": f"{prec} call (prologue + attention) + fbcache_gate"}
+        h8 = _src_hash("attn_kernel.cuh", "dit_device.cuh", "attn_fp8.cu")
+        tr8 = NCU_TRAFFIC.get(("attn_fp8_i8qk" if prec == "fp8_i8qk" else "attn_fp8", h8))
+        fp8_objs[prec]["attention_kernel_traffic"] = tr8
+        fp8_objs[prec]["traffic_source"] = (f"ncu capture of this kernel source (hash {h8})" if tr8 is not None
+                                            else f"no capture of this kernel source (hash {h8})")
         assert dit.read_error() == 0
     fp8 = fp8_objs.get("fp8_i8qk")
     fp8_e4m3 = fp8_objs.get("fp8")

@@ -433,8 +433,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
-      int j = 1;
-      for (; ok && j <= nkv; ++j) {
+      for (int j = 1; ok && j <= nkv; ++j) {
         const int jj = j - 1, sv = jj % NV, sk = j % NK;
         // another role gave up: stop issuing.  Then TMA readiness, while the
         // softmax warpgroups are still busy
@@ -485,9 +484,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         __syncwarp();
       }
-      // Failure path: the rest of the named-barrier schedule, no MMAs (out of line:
-      // inline, its loop cost the normal path 6 % of the cycles in BF16, measured)
-      if (!ok) mma_warp_finish_schedule<C::kSplitP>(j, nkv, mma_done, leader);
+      // Failure path: the rest of the named-barrier schedule, no MMAs, from the first
+      // iteration not completed: the one after the last progress published for
+      // warpgroup 1.  (Carrying the loop index out of the loop instead cost the
+      // normal path 6 % of its cycles in BF16, measured.)
+      if (!ok) mma_warp_finish_schedule<C::kSplitP>(flag_load(mma_done + 4) + 1, nkv, mma_done, leader);
    }
   } else {
     regs_inc<C::kRegsSoftmax>();

@@ -9,7 +9,7 @@
 // Cache-DiT on the TensorRT-LLM VisualGen page).
 //
 // HBM-bound: 4 bytes read per element, ~3 flops.  Pass 1 streams both inputs
-// with 16-byte loads (4 per input in flight per thread) over up to 1184 CTAs, fp32 per-thread partials,
+// with 16-byte loads (4 per input in flight per thread) over up to 740 CTAs, fp32 per-thread partials,
 // fp64 per-CTA combine; pass 2 (one CTA) combines the CTA partials in a fixed
 // tree order, so the result is deterministic for a given n.  For a residual split
 // across ranks, gate_pass2_sums stops at the two totals (summed across ranks by
@@ -25,7 +25,10 @@
 namespace dit {
 
 constexpr int kGateThreads = 256;
-constexpr int kGateMaxCtas = 148 * 8;
+// Pass 1 runs at most one wave: at 48 registers a thread, five 256-thread CTAs
+// fit on an SM, so 148 x 5 CTAs are resident at once (eight per SM would need a
+// second, partial wave; measured 5 % slower on the 16896 x 3072 pair).
+constexpr int kGateMaxCtas = 148 * 5;
 
 int gate_num_ctas(int64_t n) {
   const int64_t per_cta = static_cast<int64_t>(kGateThreads) * 8;

@@ -53,41 +53,24 @@ struct RopeArgs {
   const int32_t* skip;  // non-null and set: do nothing
 };
 
-// One thread per 8 consecutive channels (4 pairs): one 16-byte load of x, two
-// 16-byte loads of the tables, one 16-byte (bf16) or two (fp32) stores.
-// Consecutive threads walk consecutive 16-byte chunks of a token row; the grid
-// covers every chunk once (measured faster than a grid-stride loop or several
-// chunks per thread, which cost occupancy).
-__global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
-  if (a.skip != nullptr && *a.skip != 0) return;
-  const RopeJob& jb = a.job[blockIdx.y];
-  const int cpr = a.d / 8;  // chunks per row
-  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.N * cpr;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const int c = static_cast<int>(idx % cpr);
-  const int64_t row = idx / cpr;
-  const int n = static_cast<int>(row % a.N);
-  const int64_t bh = row / a.N;
-  const int h = static_cast<int>(bh % a.H);
-  const int b = static_cast<int>(bh / a.H);
-  const int64_t xo = b * jb.sx[0] + h * jb.sx[1] + n * jb.sx[2] + c * 8;
-  const int64_t yo = b * jb.sy[0] + h * jb.sy[1] + n * jb.sy[2] + c * 8;
-  const uint4 xv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(jb.x) + xo);
-  const float4 cv = *reinterpret_cast<const float4*>(a.cos_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
-  const float4 sv = *reinterpret_cast<const float4*>(a.sin_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
+// One thread per (batch, token, 8-channel chunk): it loads that chunk's cos and
+// sin (16 bytes each) once and applies them to every head, four heads at a time
+// (four independent 16-byte loads of x in flight per thread).  Consecutive
+// threads walk consecutive 16-byte chunks of a token row, so for one head a
+// warp reads 512 contiguous bytes.
+__device__ __forceinline__ void rope8(const uint4& xv, const float (&cc)[4], const float (&ss)[4], float (&y)[8]) {
   const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xv);
-  const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-  const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
-  float y[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 x2 = __bfloat1622float2(xp[i]);
     y[2 * i] = x2.x * cc[i] - x2.y * ss[i];
     y[2 * i + 1] = x2.x * ss[i] + x2.y * cc[i];
   }
-  if (a.out_fp32) {
-    float4* yp = reinterpret_cast<float4*>(static_cast<float*>(jb.y) + yo);
+}
+
+__device__ __forceinline__ void store8(void* base, int64_t off, const float (&y)[8], int out_fp32) {
+  if (out_fp32) {
+    float4* yp = reinterpret_cast<float4*>(static_cast<float*>(base) + off);
     yp[0] = make_float4(y[0], y[1], y[2], y[3]);
     yp[1] = make_float4(y[4], y[5], y[6], y[7]);
   } else {
@@ -96,7 +79,43 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
     o.y = pack_bf16x2(y[2], y[3]);
     o.z = pack_bf16x2(y[4], y[5]);
     o.w = pack_bf16x2(y[6], y[7]);
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(jb.y) + yo) = o;
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + off) = o;
+  }
+}
+
+__global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
+  if (a.skip != nullptr && *a.skip != 0) return;
+  const RopeJob& jb = a.job[blockIdx.y];
+  const int cpr = a.d / 8;  // chunks per row
+  const int64_t total = static_cast<int64_t>(a.B) * a.N * cpr;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int c = static_cast<int>(idx % cpr);
+  const int64_t row = idx / cpr;
+  const int n = static_cast<int>(row % a.N);
+  const int b = static_cast<int>(row / a.N);
+  const float4 cv = *reinterpret_cast<const float4*>(a.cos_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
+  const float4 sv = *reinterpret_cast<const float4*>(a.sin_tab + static_cast<int64_t>(n) * (a.d / 2) + c * 4);
+  const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+  const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(jb.x) + b * jb.sx[0] + n * jb.sx[2] + c * 8;
+  const int64_t yo = b * jb.sy[0] + n * jb.sy[2] + c * 8;
+  int h = 0;
+  for (; h + 4 <= a.H; h += 4) {
+    uint4 xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) xv[u] = *reinterpret_cast<const uint4*>(x + (h + u) * jb.sx[1]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float y[8];
+      rope8(xv[u], cc, ss, y);
+      store8(jb.y, yo + (h + u) * jb.sy[1], y, a.out_fp32);
+    }
+  }
+  for (; h < a.H; ++h) {
+    float y[8];
+    rope8(*reinterpret_cast<const uint4*>(x + h * jb.sx[1]), cc, ss, y);
+    store8(jb.y, yo + h * jb.sy[1], y, a.out_fp32);
   }
 }
 
@@ -108,7 +127,7 @@ cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int 
   a.B = B; a.H = H; a.N = N; a.d = d;
   a.cos_tab = cos_tab; a.sin_tab = sin_tab; a.out_fp32 = out_fp32;
   a.skip = skip;
-  const int64_t total = static_cast<int64_t>(B) * H * N * (d / 8);
+  const int64_t total = static_cast<int64_t>(B) * N * (d / 8);  // threads: one per (b, n, chunk), all heads
   const int64_t blocks = (total + 255) / 256;
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;  // grid.x limit; nothing launched
   dim3 grid(static_cast<unsigned>(blocks), njobs);

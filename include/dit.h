@@ -243,10 +243,10 @@ DIT_API dit_status fbcache_gate_ref_update(const void* r_cur, void* r_ref, int64
  * library device memory, e.g. a plug-in run by a host framework that owns the
  * device allocator, or a step loop that must not allocate while it runs.
  * Same inputs, outputs, arithmetic and result as fbcache_gate; its scratch
- * is a fixed device array of 2 * 1184 doubles (18,944 bytes) inside the
+ * is a fixed device array of 2 * 740 doubles (11,840 bytes) inside the
  * library, held by every device that loads it until the process exits.
  * Limit: the scratch must hold 2 doubles per pass-1 CTA; the CTA count is
- * capped at 1184 for any n, so every n >= 1 fits (a larger need would return
+ * capped at 740 for any n, so every n >= 1 fits (a larger need would return
  * DIT_ERR_WORKSPACE).  Nothing in the array has to start at zero.  The first
  * call on a device looks up the array's device address (a runtime query), so
  * make that first call before capturing the stream.  All calls share the one

@@ -281,7 +281,10 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
                 mma_done[i] = j
             j += 1
         if not ok and mistake != "mma_leaves_without_schedule":
-            for jd in range(j, nkv + 1):  # the rest of the named-barrier schedule, no MMAs
+            # the rest of the named-barrier schedule, no MMAs, from the iteration after
+            # the last one whose progress was published for warpgroup 1
+            assert mma_done[1] + 1 == j
+            for jd in range(mma_done[1] + 1, nkv + 1):
                 for i in range(2):
                     if split:
                         yield named_sync(p_half[i], "mma", 32)
