@@ -503,6 +503,15 @@ def run_ours(args, rank, world, local_rank):
             "fp8_e4m3": fp8_e4m3,
             "side_kernels": side,
             "sm_mcycles_per_step": mcycles(ms_per_step, clocks),
+            "accuracy": {
+                "bf16": "max-abs <= 2e-2 and cosine >= 0.9999 against exact attention on the bf16-rounded rotated "
+                        "Q and K; against the exact-rotation oracle cosine >= 0.9999 but max-abs 0.08-0.15 on the "
+                        "outlier-channel workloads (the bf16 rounding of the rotated operands alone)",
+                "fp8_i8qk": "cosine ~0.998 against exact attention on the x8 outlier-channel Flux workloads "
+                            "(target 0.995); ~0.999 on N(0,1) inputs",
+                "fp8_e4m3": "cosine ~0.978 against exact attention on the outlier workloads (the e4m3 Q.K^T floor); "
+                            "~0.9986 on N(0,1) inputs",
+                "how": "pytest -m gpu (tests/test_gpu_attention.py, tests/test_gpu_fp8.py)"},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": max(all_e2e) / ke,
