@@ -28,10 +28,17 @@
 // FP8: Q, K and V arrive rotated, smoothed (K) and quantised from one prologue
 // pass (rotating and quantising Q here measured 4 % slower per tile).
 // TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256) O0, O1 (d
-// columns each from 256).  P_i (bf16: 64 columns, e4m3: 32) overwrites the
-// first columns of S_i once the softmax has read S_i.
-// The MMA thread issues, per key tile j:
+// columns each from 256).  BF16: P_i (64 columns of bf16 pairs) overwrites the
+// first columns of S_i once the softmax has read S_i.  FP8: P_i is written to
+// a shared-memory tile of its own (see kPSmem), and S_i is free as soon as the
+// softmax has loaded it into registers.
+// The BF16 MMA thread issues, per key tile j:
 //     O0 += P0(j-1) V(j-1);  S0(j) = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1(j) = Q1 K(j)^T
+// The FP8 MMA thread issues, per key tile j:
+//     S0(j) (once softmax 0 has read S0(j-1));  S1(j) (likewise);
+//     O0 += P0(j-1) V(j-1);  O1 += P1(j-1) V(j-1)
+// and commits each PV to pv_done_i, which softmax i waits for before it
+// overwrites P_i or rescales O_i.  (The ordering argument below is BF16's.)
 // tcgen05 MMAs from one thread are executed in issue order, so S_i(j) never
 // overwrites P_i(j-1) before PV_i(j-1) has read it, and a tcgen05.commit
 // tracks every MMA the thread issued before it: when softmax i sees S_i(j)
@@ -69,8 +76,16 @@ struct AttnCfg {
   static constexpr int kBoxInner = 128 / EB;            // TMA box inner extent (elements)
   static constexpr int NK = (!FP8 && D == 128) ? 3 : 4;
   static constexpr int NV = (!FP8 && D == 128) ? 2 : 4;
-  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1;
-  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + kNumBars * 8 + 32;
+  // FP8: P_i goes to shared memory (one [128 rows][128 keys] e4m3 tile per Q
+  // tile, the same 128-byte-swizzled K-major layout as a Q tile) instead of
+  // overwriting S_i in TMEM, so S_i(j+1) may be computed as soon as softmax i
+  // has read S_i(j) into registers: the softmax never waits for PV_i(j) and
+  // S_i(j+1) to run back to back.  BF16's P (32 KB per tile) does not fit.
+  static constexpr bool kPSmem = FP8;
+  static constexpr int kPTileBytes = kPSmem ? BM * BN : 0;
+  static constexpr int kNumBars = 2 + 2 * NK + 2 * NV + 2 + 2 + 2 + 1 + 2 + 2;
+  static constexpr int kSmemBytes =
+      1024 + 2 * kTileBytes + (NK + NV) * kTileBytes + 2 * kPTileBytes + kNumBars * 8 + 32;
   static constexpr int kKStep = FP8 ? 32 : 16;          // K extent of one MMA (elements)
   static constexpr uint32_t kColS = 0, kColO = 256;     // S_i at 128 i, O_i at 256 + D i
   static constexpr uint32_t kTmemCols = 512;
@@ -248,15 +263,19 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* sQ = smem;                        // Q0, Q1
   uint8_t* sK = sQ + 2 * C::kTileBytes;      // NK stages
   uint8_t* sV = sK + NK * C::kTileBytes;     // NV stages
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(sV + NV * C::kTileBytes);  // [2]
+  uint8_t* sP = sV + NV * C::kTileBytes;     // FP8: P0, P1
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + 2 * C::kPTileBytes);  // [2]
   uint64_t* k_full = q_full + 2;
   uint64_t* k_empty = k_full + NK;
   uint64_t* v_full = k_empty + NK;
   uint64_t* v_empty = v_full + NV;
   uint64_t* s_full = v_empty + NV;   // [2] S_i(j) computed (and every earlier MMA)
-  uint64_t* pv_done = s_full + 2;    // [2] the last PV_i computed (read by the epilogue)
+  uint64_t* pv_done = s_full + 2;    // [2] BF16: the last PV_i computed (read by the epilogue);
+                                     //     FP8: every PV_i(j) computed (one phase per tile)
   uint64_t* q_ready = pv_done + 2;   // [2] BF16: Q_i rotated in shared memory (128 arrivals)
   uint64_t* mma_drain = q_ready + 2; // failure path: every MMA the MMA thread issued has completed
+  uint64_t* s_free = mma_drain + 1;  // [2] FP8: softmax i has read S_i(j) (one arrival per warp)
+  uint64_t* p_ready = s_free + 2;    // [2] FP8: softmax i has stored P_i(j) (one arrival per warp)
   // named barriers: kBarPReady + i  softmax i finished tile j (128 arrive, MMA warp syncs)
   //                 kBarTurn + i    softmax i may exponentiate (128 arrive, 128 sync)
   //                 kBarPHalf + i   BF16: softmax i stored keys 0..63 of P (128 arrive, MMA warp syncs)
@@ -295,6 +314,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(s_full + i, 1);
       mbar_init(pv_done + i, 1);
       mbar_init(q_ready + i, 128);
+      mbar_init(s_free + i, 4);
+      mbar_init(p_ready + i, 4);
     }
     for (int s = 0; s < NK; ++s) {
       mbar_init(k_full + s, 1);
@@ -376,6 +397,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
+      const uint32_t p_addr = smem_u32(sP);
       auto qk = [&](int i, int sk) {  // S_i = Q_i K^T
         const uint32_t qa = q_addr + i * C::kTileBytes, ka = k_addr + sk * C::kTileBytes;
         // S_i's columns end before O's; the K stage is one of the ring's
@@ -398,17 +420,23 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t va = v_addr + sv * C::kTileBytes;
         // O_i inside the allocation, P inside S_i, the V stage one of the ring's
         if (!debug_check(i < 2 && sv < NV && C::kColO + D * (i + 1) <= C::kTmemCols && k1 * 8 <= BN &&
-                             k0 >= 0, err))
+                             k0 >= 0 && (!C::kPSmem || k1 * 32 <= BN), err))
           return;
 #pragma unroll
         for (int kk = k0; kk < k1; ++kk) {
           // kKStep keys = kKStep rows of 128 bytes; d column blocks are kSubBytes apart
           const uint64_t bd = smem_desc_sw128(va + kk * C::kKStep * 128, C::kSubBytes, 1024);
-          const uint32_t pa = tmem + C::kColS + 128 * i + kk * 8;  // 8 columns of packed P per MMA
-          if constexpr (FP8)
-            mma_f8_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
-          else
-            mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
+          if constexpr (C::kPSmem) {
+            // P_i in shared memory, K-major like a Q tile: kKStep keys = 32 bytes of each row
+            const uint64_t ad = smem_desc_sw128(p_addr + i * C::kPTileBytes + kk * 32, 16, 1024);
+            mma_f8_ss(tmem + C::kColO + D * i, ad, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
+          } else {
+            const uint32_t pa = tmem + C::kColS + 128 * i + kk * 8;  // 8 columns of packed P per MMA
+            if constexpr (FP8)
+              mma_f8_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
+            else
+              mma_f16_ts(tmem + C::kColO + D * i, pa, bd, idesc_o, (acc || kk > k0) ? 1u : 0u);
+          }
         }
       };
       const bool leader = lane == 0;
@@ -433,7 +461,61 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
-      for (int j = 1; ok && j <= nkv; ++j) {
+      if constexpr (C::kPSmem) {
+        // FP8: lane 0 polls four event streams and issues whatever is ready, so that
+        // neither softmax warpgroup waits behind the other's hand-offs:
+        //   S_i(ns_i)  once softmax i has read S_i(ns_i - 1) and K(ns_i) has landed
+        //   PV_i(np_i) once softmax i has stored P_i(np_i) and V(np_i) has landed
+        // Each barrier is at most one phase ahead of the parity polled (the next
+        // phase needs the MMA being waited for), so every poll is unambiguous.
+        // Bounded: it gives up when another role raised the abort flag, or after
+        // kWaitLimitNs without progress (recording the timeout and raising the flag).
+        if (leader && ok) {
+          int ns[2] = {1, 1}, np[2] = {0, 0};
+          uint32_t idle = 0;
+          uint64_t idle_since = 0;
+          while (np[0] < nkv || np[1] < nkv) {
+            bool progress = false;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int js = ns[i], sk = js % NK;
+              if (js < nkv && mbar_try_wait(smem_u32(s_free + i), (js - 1) & 1) &&
+                  mbar_try_wait(smem_u32(k_full + sk), (js / NK) & 1)) {
+                tc_fence_after();
+                qk(i, sk);
+                mma_commit(s_full + i);
+                mma_commit(k_empty + sk);
+                ns[i] = js + 1;
+                progress = true;
+              }
+              const int jp = np[i], sv = jp % NV;
+              if (jp < nkv && mbar_try_wait(smem_u32(p_ready + i), jp & 1) &&
+                  mbar_try_wait(smem_u32(v_full + sv), (jp / NV) & 1)) {
+                tc_fence_after();
+                pv(i, sv, jp > 0, 0, BN / C::kKStep);
+                mma_commit(pv_done + i);  // P_i may be overwritten, O_i rescaled or read
+                mma_commit(v_empty + sv);
+                np[i] = jp + 1;
+                progress = true;
+              }
+            }
+            if (progress) {
+              idle = 0;
+            } else if ((++idle & 63u) == 1u) {
+              const uint64_t now = globaltimer_ns();
+              if (idle == 1u) idle_since = now;
+              if (flag_load(abort_flag) != 0) break;
+              if (now - idle_since > kWaitLimitNs) {
+                set_error(err, kErrTimeout);
+                flag_store(abort_flag, 1);
+                break;
+              }
+            }
+          }
+        }
+        __syncwarp();
+      }
+      for (int j = 1; !C::kPSmem && ok && j <= nkv; ++j) {
         const int jj = j - 1, sv = jj % NV, sk = j % NK;
         // another role gave up: stop issuing.  Then TMA readiness, while the
         // softmax warpgroups are still busy
@@ -443,6 +525,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         constexpr int NKK = BN / C::kKStep, KH = C::kSplitP ? NKK / 2 : 0;
+
         if constexpr (C::kSplitP) {  // first half of PV_0 while softmax 0 finishes P_0
           named_sync<kBarPHalf + 0, 160>();
           tc_fence_after();
@@ -488,7 +571,7 @@ __global__ void __launch_bounds__(384, 1)
       // iteration not completed: the one after the last progress published for
       // warpgroup 1.  (Carrying the loop index out of the loop instead cost the
       // normal path 6 % of its cycles in BF16, measured.)
-      if (!ok) mma_warp_finish_schedule<C::kSplitP>(flag_load(mma_done + 4) + 1, nkv, mma_done, leader);
+      if (!C::kPSmem && !ok) mma_warp_finish_schedule<C::kSplitP>(flag_load(mma_done + 4) + 1, nkv, mma_done, leader);
    }
   } else {
     regs_inc<C::kRegsSoftmax>();
@@ -583,6 +666,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_wait_ld();
       reg_fence(s);
+      if constexpr (C::kPSmem) {  // S_i is in registers: the MMA warp may compute S_i(j+1) into it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + i);
+      }
       if constexpr (I8QK) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) s[c] = s32_biased_f32(s[c]);
@@ -675,7 +763,7 @@ __global__ void __launch_bounds__(384, 1)
             acc[2 * (q >> 1) + 1] = fadd2(acc[2 * (q >> 1) + 1], f2(cc, dd));
             p[8 * q + e] = cvt_e4m3x4(a, bq, cc, dd);
           }
-          tmem_st8(tS + 8 * q, p + 8 * q);
+          if constexpr (!C::kPSmem) tmem_st8(tS + 8 * q, p + 8 * q);
         } else {  // 32 keys -> 16 columns of 2 bf16
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -709,12 +797,34 @@ __global__ void __launch_bounds__(384, 1)
         if (i == 0) named_arrive<kBarTurn + 1, 256>();
         else if (j + 1 < nkv) named_arrive<kBarTurn + 0, 256>();
       }
-      tmem_wait_st();
-      reg_fence(p);
+      if constexpr (C::kPSmem) {
+        // PV_i(j-1) has read P_i and finished writing O_i: then P_i(j) replaces it
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, (j - 1) & 1, err, kErrTimeout, abort_flag));
+          if (!ok) break;
+        }
+        // row `row`, 16-byte chunk c (keys 16c..16c+15) at slot c ^ (row % 8) of the row's 128 bytes
+        uint8_t* prow = sP + i * C::kPTileBytes + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (debug_check(i * C::kPTileBytes + row * 128 + 128 <= 2 * C::kPTileBytes, err))
+            st_shared_v4(prow + ((c ^ (row & 7)) << 4), p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+        // the MMA reads P through the async proxy: order the generic-proxy writes first
+        fence_proxy_async_smem();
+      } else {
+        tmem_wait_st();
+        reg_fence(p);
+      }
       if (!C::kSplitP && j > 0 && grow) rescale_o(alpha);
       tc_fence_before();
-      if (i == 0) named_arrive<kBarPReady + 0, 160>();
-      else named_arrive<kBarPReady + 1, 160>();
+      if constexpr (C::kPSmem) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_ready + i);
+      } else if (i == 0) {
+        named_arrive<kBarPReady + 0, 160>();
+      } else {
+        named_arrive<kBarPReady + 1, 160>();
+      }
       float a0, a1;
       if constexpr (FP8) {  // divide each half's V block scale back out of its row sum
         float b0, b1;
@@ -727,7 +837,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       m = m_new;
     }
-    if (!ok) {
+    if (!C::kPSmem && !ok) {
       // Failure path: the rest of this warpgroup's named-barrier schedule (tiles j..nkv-1)
       // without the work between, so the MMA warp and the other warpgroup are never
       // left waiting on an arrival from here.  Each arrival waits (bounded) until the
@@ -758,7 +868,9 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, 0, err, kErrTimeout, abort_flag));
+    // BF16 commits pv_done once, after the last PV; FP8 once per tile
+    const uint32_t pv_last = C::kPSmem ? static_cast<uint32_t>((nkv - 1) & 1) : 0u;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + i, pv_last, err, kErrTimeout, abort_flag));
     if (ok) {
       tc_fence_after();
       const float fin = fin_scale / l;

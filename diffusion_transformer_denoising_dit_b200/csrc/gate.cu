@@ -11,7 +11,10 @@
 // HBM-bound: 4 bytes read per element, ~3 flops.  Pass 1 streams both inputs
 // with 16-byte loads (4 per input in flight per thread) over up to 740 CTAs, fp32 per-thread partials,
 // fp64 per-CTA combine; pass 2 (one CTA) combines the CTA partials in a fixed
-// tree order, so the result is deterministic for a given n.  For a residual split
+// order, so the result is deterministic for a given n.  Pass 2 is a programmatic
+// dependent launch: it is scheduled while pass 1 still runs and waits on the
+// device (griddepcontrol.wait) until pass 1 has completed and its partials are
+// visible, so no launch gap separates the two.  For a residual split
 // across ranks, gate_pass2_sums stops at the two totals (summed across ranks by
 // the caller) and gate_finalize takes the decision from the summed totals.
 #include <cuda_bf16.h>
@@ -53,6 +56,8 @@ __device__ __forceinline__ void accum8(const uint4& av, const uint4& bv, float& 
 __global__ void __launch_bounds__(kGateThreads) gate_pass1(const __nv_bfloat16* __restrict__ a,
                                                            const __nv_bfloat16* __restrict__ b, int64_t n,
                                                            double* __restrict__ partials) {
+  // the dependent combine may be scheduled now; it waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   float num = 0.f, den = 0.f;
   const int64_t n8 = n / 8;
   const uint4* a8 = reinterpret_cast<const uint4*>(a);
@@ -102,24 +107,37 @@ __global__ void __launch_bounds__(kGateThreads) gate_pass1(const __nv_bfloat16* 
   }
 }
 
-// The per-CTA partials combined in a fixed tree order (one 1024-thread CTA);
-// the totals land in sn[0], sd[0].
-__device__ __forceinline__ void combine_partials(const double* __restrict__ partials, int nparts, double* sn,
-                                                 double* sd) {
-  double tn = 0.0, td = 0.0;
-  for (int k = threadIdx.x; k < nparts; k += blockDim.x) {
-    tn += partials[2 * k];
-    td += partials[2 * k + 1];
+constexpr int kCombineThreads = 256;
+
+// The per-CTA partials combined in a fixed order by one kCombineThreads CTA:
+// thread t sums partials t, t + 256, ... in turn, each warp folds its 32 sums
+// with a butterfly, and thread 0 adds the 8 warp sums in warp order.  Returns
+// the totals in thread 0.
+__device__ __forceinline__ void combine_partials(const double* __restrict__ partials, int nparts, double& tn,
+                                                 double& td) {
+  double n = 0.0, d = 0.0;
+  for (int k = threadIdx.x; k < nparts; k += kCombineThreads) {
+    n += partials[2 * k];
+    d += partials[2 * k + 1];
   }
-  sn[threadIdx.x] = tn;
-  sd[threadIdx.x] = td;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n += __shfl_xor_sync(0xffffffffu, n, o);
+    d += __shfl_xor_sync(0xffffffffu, d, o);
+  }
+  __shared__ double sn[kCombineThreads / 32], sd[kCombineThreads / 32];
+  if ((threadIdx.x & 31) == 0) {
+    sn[threadIdx.x >> 5] = n;
+    sd[threadIdx.x >> 5] = d;
+  }
   __syncthreads();
-  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
-    if (threadIdx.x < s) {
-      sn[threadIdx.x] += sn[threadIdx.x + s];
-      sd[threadIdx.x] += sd[threadIdx.x + s];
+  tn = 0.0, td = 0.0;
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) {
+      tn += sn[w];
+      td += sd[w];
     }
-    __syncthreads();
   }
 }
 
@@ -134,23 +152,45 @@ __device__ __forceinline__ void decide(double num, double den, float threshold, 
   skip_out[0] = (rel < static_cast<double>(threshold)) ? 1 : 0;
 }
 
-__global__ void __launch_bounds__(1024) gate_pass2(const double* __restrict__ partials, int nparts, float threshold,
-                                                   float* __restrict__ rel_out, int32_t* __restrict__ skip_out) {
-  __shared__ double sn[1024], sd[1024];
-  combine_partials(partials, nparts, sn, sd);
-  if (threadIdx.x == 0) decide(sn[0], sd[0], threshold, rel_out, skip_out);
+// griddepcontrol.wait: pass 1 has completed and its partials are visible (a
+// no-op when this grid was launched without the programmatic dependency)
+__global__ void __launch_bounds__(kCombineThreads) gate_pass2(const double* __restrict__ partials, int nparts,
+                                                              float threshold, float* __restrict__ rel_out,
+                                                              int32_t* __restrict__ skip_out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  double tn, td;
+  combine_partials(partials, nparts, tn, td);
+  if (threadIdx.x == 0) decide(tn, td, threshold, rel_out, skip_out);
 }
 
 // Sharded form: the shard's totals (sum |a - b|, sum |b|) in fp64, to be summed
 // across ranks before gate_finalize decides.
-__global__ void __launch_bounds__(1024) gate_pass2_sums(const double* __restrict__ partials, int nparts,
-                                                        double* __restrict__ sums_out) {
-  __shared__ double sn[1024], sd[1024];
-  combine_partials(partials, nparts, sn, sd);
+__global__ void __launch_bounds__(kCombineThreads) gate_pass2_sums(const double* __restrict__ partials, int nparts,
+                                                                   double* __restrict__ sums_out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  double tn, td;
+  combine_partials(partials, nparts, tn, td);
   if (threadIdx.x == 0) {
-    sums_out[0] = sn[0];
-    sums_out[1] = sd[0];
+    sums_out[0] = tn;
+    sums_out[1] = td;
   }
+}
+
+// Launches a one-CTA combine as a programmatic dependent of the kernel before it
+// on the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 __global__ void gate_finalize(const double* __restrict__ sums, float threshold, float* __restrict__ rel_out,
@@ -165,8 +205,7 @@ cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold
                                              static_cast<const __nv_bfloat16*>(b), n, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gate_pass2<<<1, 1024, 0, stream>>>(partials, g, threshold, rel_out, skip_out);
-  return cudaGetLastError();
+  return launch_dependent(gate_pass2, stream, static_cast<const double*>(partials), g, threshold, rel_out, skip_out);
 }
 
 cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* sums_out, double* partials,
@@ -176,8 +215,7 @@ cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* su
                                              static_cast<const __nv_bfloat16*>(b), n, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gate_pass2_sums<<<1, 1024, 0, stream>>>(partials, g, sums_out);
-  return cudaGetLastError();
+  return launch_dependent(gate_pass2_sums, stream, static_cast<const double*>(partials), g, sums_out);
 }
 
 cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,

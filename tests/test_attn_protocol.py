@@ -7,8 +7,12 @@ a TMA producer, an MMA issuer and two softmax warpgroups, linked by mbarriers
 buffer overwritten too early is a silent wrong answer, so the protocol is
 modelled here step by step as the kernel performs it and run under many random
 interleavings, with the kernel's three configurations (BF16 d=128: K ring 3, V
-ring 2, P handed over in two halves, ping-pong turns; BF16 d=64: rings 4/4;
-FP8: rings 4/4, whole P, no turns).
+ring 2, P handed over in two halves in TMEM, ping-pong turns; BF16 d=64: rings
+4/4; FP8: rings 4/4, no turns and no named barriers: P in a shared-memory tile
+of its own, handed over through a p_ready mbarrier; the MMA thread polls four
+event streams and issues S_i(j) once softmax i has read S_i(j-1) and PV_i(j)
+once P_i(j) is stored, whichever is ready first; every PV is committed to
+pv_done, which softmax i waits for before it overwrites P_i or rescales O_i).
 
 Semantics modelled:
 * mbarrier: a phase completes after `count` arrivals; a parity wait succeeds
@@ -28,8 +32,10 @@ Semantics modelled:
 Checks: no deadlock; every role finishes; an MMA reads the K/V tile, the Q tile
 (rotated, for BF16) and the half of P it was issued for; no TMA load lands in a
 stage an issued MMA still reads; the softmax reads S and writes P only while no
-issued MMA touches that half of the buffer; O is rescaled and read only while
-no PV into it is outstanding; nothing is in flight when the CTA ends.  Planted
+issued MMA touches that half of the buffer (FP8: reads S while no S MMA of its
+tile is outstanding, writes its P tile while no PV reads it); O is rescaled and
+read only while no PV into it is outstanding; nothing is in flight when the
+CTA ends.  Planted
 protocol mistakes (negative controls) must each be caught.
 
 Failure path (as in the kernel): every mbarrier wait is bounded; the first one
@@ -108,6 +114,7 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
     """
     rng = random.Random(seed)
     split = pingpong = not fp8
+    psmem = fp8  # P in shared memory, S freed once read
     errors = []
     q_full = [MBar(1), MBar(1)]
     q_ready = [MBar(1), MBar(1)]  # 128 arrivals in the kernel: one per softmax thread, modelled as one
@@ -117,6 +124,8 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
     v_empty = [MBar(2) for _ in range(NV)]
     s_full = [MBar(1), MBar(1)]
     pv_done = [MBar(1), MBar(1)]
+    s_free = [MBar(1), MBar(1)]  # FP8: one arrival per softmax warp in the kernel, modelled as one
+    p_ready_m = [MBar(1), MBar(1)]  # FP8: likewise
     bars = {"s_full": s_full, "pv_done": pv_done, "k_empty": k_empty, "v_empty": v_empty}
     p_ready = [Named(f"PReady{i}", 160, errors) for i in range(2)]
     p_half = [Named(f"PHalf{i}", 160, errors) for i in range(2)]
@@ -130,6 +139,7 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
     qstate = ["none", "none"]
     kstage, vstage = {}, {}
     buf = [[None, None], [None, None]]  # S_i buffer halves: ("S", j) or ("P", j)
+    psm = [None, None]                  # FP8: P_i shared-memory tile, ("P", j)
     tma = []                            # loads in flight: (kind, slot, tile)
     queue, issued, completed = [], [0], [0]
     commits = []                        # (MMAs that must have completed, barrier)
@@ -162,6 +172,9 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
     def touching(i, half):
         return [m for m in queue if m["i"] == i and (m["kind"] == "S" or half in m["halves"])]
 
+    def s_pending(i):
+        return any(m["kind"] == "S" and m["i"] == i for m in queue)
+
     def pv_pending(i):
         return any(m["kind"] == "PV" and m["i"] == i for m in queue)
 
@@ -178,9 +191,13 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
         else:
             if vstage.get(m["stage"]) != j:
                 errors.append(f"PV{i}({j}) read V stage {m['stage']} holding {vstage.get(m['stage'])}")
-            for h in m["halves"]:
-                if buf[i][h] != ("P", j):
-                    errors.append(f"PV{i}({j}) read half {h} holding {buf[i][h]}")
+            if psmem:
+                if psm[i] != ("P", j):
+                    errors.append(f"PV{i}({j}) read the P tile holding {psm[i]}")
+            else:
+                for h in m["halves"]:
+                    if buf[i][h] != ("P", j):
+                        errors.append(f"PV{i}({j}) read half {h} holding {buf[i][h]}")
         completed[0] += 1
         fire_commits()
 
@@ -251,6 +268,42 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
             issue("S", 1, 0, 0, halves_all)
             commit("s_full", 1)
             commit("k_empty", 0)
+        if psmem:
+            # event-driven: each pass issues every S and PV whose inputs are ready
+            ns, npv = [1, 1], [0, 0]
+
+            def s_ready(i):
+                t = ns[i]
+                return (t < nkv and (mistake == "s_before_read" or s_free[i].done((t - 1) & 1))
+                        and k_full[t % NK].done((t // NK) & 1))
+
+            def pv_ready(i):
+                t = npv[i]
+                return t < nkv and p_ready_m[i].done(t & 1) and v_full[t % NV].done((t // NV) & 1)
+
+            while ok and (npv[0] < nkv or npv[1] < nkv):
+                cond = lambda: any(s_ready(i) or pv_ready(i) for i in range(2))
+                if mistake == "mma_poll_unbounded":
+                    yield cond
+                else:
+                    ok = yield ("mbar", cond)
+                if not ok:
+                    break
+                for i in range(2):
+                    if s_ready(i):
+                        t = ns[i]
+                        issue("S", i, t, t % NK, halves_all)
+                        commit("s_full", i)
+                        commit("k_empty", t % NK)
+                        ns[i] += 1
+                    if pv_ready(i):
+                        t = npv[i]
+                        issue("PV", i, t, t % NV, halves_all)
+                        commit("pv_done", i)
+                        commit("v_empty", t % NV)
+                        npv[i] += 1
+                    yield lambda: True  # other roles run between the checks
+            return
         j = 1
         while ok and j <= nkv:
             jj, sv, sk = j - 1, (j - 1) % NV, j % NK
@@ -306,9 +359,28 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
             ok = yield ("mbar", lambda j=j: s_full[i].done(j & 1))
             if not ok:
                 break
-            if any(m["kind"] == "S" and m["i"] == i for m in queue) or buf[i] != [("S", j), ("S", j)]:
+            if s_pending(i) or buf[i] != [("S", j), ("S", j)]:
                 errors.append(f"softmax{i}({j}) reads S holding {buf[i]} with MMAs {len(queue)} in flight")
             grow = j > 0 and rng.random() < 0.5
+            if psmem:
+                s_free[i].arrive()  # S_i is in registers
+                yield lambda: True  # the exponentials: anything may run meanwhile
+                if j > 0 and mistake != "p_store_without_pv_wait":
+                    ok = yield ("mbar", lambda j=j: pv_done[i].done((j - 1) & 1))
+                    if not ok:
+                        break
+                if pv_pending(i):
+                    errors.append(f"softmax{i}({j}) writes its P tile while a PV reads it")
+                psm[i] = ("P", j)
+                if grow and mistake != "rescale_after_release" and pv_pending(i):
+                    errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
+                p_ready_m[i].arrive()
+                if grow and mistake == "rescale_after_release":
+                    yield lambda: True
+                    if pv_pending(i):
+                        errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
+                j += 1
+                continue
             if pingpong:
                 if i == 1:
                     yield named_sync(turn[1], who, 128)
@@ -336,7 +408,7 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
                 if pv_pending(i):
                     errors.append(f"softmax{i}({j}) rescales O while a PV writes it")
             j += 1
-        if not ok and mistake != "softmax_leaves_without_schedule":
+        if not ok and not psmem and mistake != "softmax_leaves_without_schedule":
             # the rest of the named-barrier schedule, no work; each arrival waits until its
             # partner has passed the previous generation (the pacing the data
             # dependencies give on the normal path), so arrivals never run a generation
@@ -366,8 +438,9 @@ def simulate(fp8, NK, NV, nkv, seed, mistake=None, lost=None, report=None):
                         turn[0].arrive(who, 128)
                 p_ready[i].arrive(who, 128)
                 yield lambda: True
-        if ok:
-            ok = yield ("mbar", lambda: pv_done[i].done(0))
+        if ok:  # BF16 commits pv_done after the last PV only, FP8 after every PV
+            last = (nkv - 1) & 1 if psmem else 0
+            ok = yield ("mbar", lambda: pv_done[i].done(last))
         if ok and pv_pending(i):
             errors.append(f"softmax{i} reads O while a PV writes it")
 
@@ -454,7 +527,8 @@ PLANTED = [
     ("k_empty_single_release", "bf16_d128"),      # K stage freed after S0 alone
     ("producer_parity_without_xor", "fp8_d128"),  # waits for the wrong phase: hangs
     ("s_before_pv", "bf16_d128"),                 # next S overwrites P before PV read it
-    ("s_before_pv", "fp8_d128"),
+    ("s_before_read", "fp8_d128"),                # next S issued before the softmax read S
+    ("p_store_without_pv_wait", "fp8_d128"),      # P tile overwritten while the last PV reads it
     ("mma_waits_unrotated_q", "bf16_d128"),       # S reads Q before its rotation
     ("rescale_after_release", "fp8_d128"),        # O rescaled after P was handed over
     ("rescale_after_release", "bf16_d64"),
@@ -477,7 +551,10 @@ def _faults(cfg):
     V), each stage release and each S / PV completion signal."""
     out = [("load", "Q", 0), ("load", "Q", 1)]
     out += [("load", kind, t) for kind in ("K", "V") for t in range(7)]
-    out += [("commit", "pv_done", 0, 0), ("commit", "pv_done", 1, 0)]
+    if cfg["fp8"]:  # one pv_done commit per tile
+        out += [("commit", "pv_done", i, n) for i in range(2) for n in (0, 3, 6)]
+    else:
+        out += [("commit", "pv_done", 0, 0), ("commit", "pv_done", 1, 0)]
     for name, n, per in (("k_empty", cfg["NK"], 2), ("v_empty", cfg["NV"], 2), ("s_full", 2, 1)):
         for idx in range(n):
             uses = 7 if name == "s_full" else -(-7 // n) * per
@@ -532,8 +609,9 @@ def test_fault_free_runs_raise_no_abort_and_leave_nothing_in_flight(name):
 # (or exits with a load in flight) under some single loss.
 FAILURE_PATH_MISTAKES = [
     ("dry_without_pacing", "bf16_d128", ("load", "Q", 0)),
-    ("dry_without_pacing", "fp8_d128", ("load", "V", 2)),
-    ("softmax_leaves_on_timeout", "fp8_d128", ("commit", "s_full", 0, 2)),
+    ("dry_without_pacing", "bf16_d64", ("load", "V", 2)),
+    ("softmax_leaves_on_timeout", "bf16_d64", ("commit", "s_full", 0, 2)),
+    ("mma_poll_unbounded", "fp8_d128", ("load", "K", 3)),      # FP8's issuer without its time limit
     ("softmax_leaves_on_timeout", "bf16_d128", ("commit", "s_full", 1, 2)),
     ("dry_schedule_without_turns", "bf16_d128", ("commit", "s_full", 0, 2)),
     ("mma_leaves_without_schedule", "bf16_d64", ("load", "V", 3)),
