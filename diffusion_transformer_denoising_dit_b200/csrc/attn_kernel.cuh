@@ -57,6 +57,8 @@
 
 #include <cuda_bf16.h>
 
+#include <cfloat>
+
 #include "dit_device.cuh"
 
 namespace dit {
@@ -151,6 +153,12 @@ __device__ __forceinline__ uint32_t s32_biased_f32(uint32_t s) {
   uint32_t r;
   asm("lop3.b32 %0, %1, 0x007FFFFF, 0x4B400000, 0x6A;" : "=r"(r) : "r"(s));
   return r;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ float lg2(float x) {
@@ -687,8 +695,11 @@ __global__ void __launch_bounds__(384, 1)
         // a half past the end keeps 1: its keys are -inf (-inf * c1 = -inf) and its p are 0
         c0 = qs * ksn0;
         c1 = qs * ksn1;
-        f0 = vsn0 * vfold;
-        f1 = vsn1 * vfold;
+        // held in the normal range, so that lg2 and the reciprocal below stay finite
+        // (a V block of denormal values then contributes nothing to P.V, as it
+        // would contribute nothing measurable to O)
+        f0 = fmaxf(vsn0 * vfold, FLT_MIN);
+        f1 = fmaxf(vsn1 * vfold, FLT_MIN);
         const int kb0 = 2 * j + 2, kb1 = 2 * j + 3;  // the next tile's blocks
         ksn0 = kb0 < nk ? ksc[kb0] : 1.f;
         vsn0 = kb0 < nk ? vsc[kb0] : 1.f;
@@ -830,7 +841,9 @@ __global__ void __launch_bounds__(384, 1)
         float b0, b1;
         f2_split(fadd2(acc[0], acc[1]), a0, a1);
         f2_split(fadd2(acc[2], acc[3]), b0, b1);
-        l = l * alpha + ((a0 + a1) * __frcp_rn(f0) + (b0 + b1) * __frcp_rn(f1));
+        // approximate reciprocals (MUFU, relative error ~2^-23): the IEEE-rounded
+        // ones cost a multi-instruction sequence twice per tile on the critical path
+        l = l * alpha + ((a0 + a1) * rcp_approx(f0) + (b0 + b1) * rcp_approx(f1));
       } else {
         f2_split(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
         l = l * alpha + (a0 + a1);

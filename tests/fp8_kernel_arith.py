@@ -9,7 +9,9 @@ computes in fp32, on the oracle's 8-bit codes and block scales:
   some row's tile max exceeds it by more than tau = 4 (log2 units);
 * P = 2^(x + log2 f - m) with f = sV(half) * 448 / (sV_max * 2^4), rounded to e4m3
   (RNE, saturating) -- the V block scale folded into the exponent;
-* row sum of the unrounded P, each half divided by its f; O rescaled by
+* row sum of the unrounded P, each half divided by its f (the kernel multiplies
+  by an approximate reciprocal, within 2^-22 relative; the model divides), f held
+  at or above FLT_MIN as the kernel holds it; O rescaled by
   2^(m_old - m_new) when the max moved; O += P8 V8; output O * sV_max * 2^4 / 448 / l.
 
 Rows are taken in groups of 32 from the start of `rows`: pass whole aligned
@@ -84,7 +86,7 @@ def kernel_model_codes(q8, k8, v8, sq, sk, sv, rows, scale=None, qk="e4m3"):
                             continue
                         sl = slice(64 * half, min(64 * (half + 1), n))
                         c[:, sl] = qs[:, None] * f32(sk[b, h][kb])
-                        f[sl] = f32(sv[b, h][kb]) * vfold
+                        f[sl] = max(f32(sv[b, h][kb]) * vfold, np.finfo(f32).tiny)
                     m_tile = (s * c).max(axis=1)
                     grow = bool((m_tile > m + f32(TAU)).any())
                     m_new = np.maximum(m, m_tile) if grow else m
