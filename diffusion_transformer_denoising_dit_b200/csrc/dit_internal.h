@@ -8,6 +8,26 @@
 
 namespace dit {
 
+// Launches `kernel` as a programmatic dependent of the grid before it on the
+// stream: it may be scheduled once every CTA of that grid has called
+// pdl_trigger (or exited), and it must call pdl_wait before it reads anything
+// that grid writes.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Keys per K/V tile of the attention kernels (the TMA box height of the K and V maps).
 constexpr int kAttnBlockN = 128;
 

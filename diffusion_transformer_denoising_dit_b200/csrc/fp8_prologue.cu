@@ -76,6 +76,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 __global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __restrict__ partial) {
+  pdl_trigger();  // the mean's combine (and through it the quantiser) may be scheduled
   const int bh = blockIdx.y;
   const int chunk = blockIdx.x;
   if (chunk == 0 && threadIdx.x == 0) p.v_scale_max[bh] = 0.f;
@@ -108,6 +109,8 @@ __global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __re
 // K channel means: one CTA per (b,h), thread c sums the kChunks partials of
 // channel c in a fixed order (independent loads, then the adds).
 __global__ void __launch_bounds__(128) kmean_finalize(Fp8Prep p, const float* __restrict__ partial) {
+  pdl_trigger();  // the quantiser may be scheduled: its Q blocks need nothing from here
+  pdl_wait();     // every partial written
   const int bh = blockIdx.x;
   const int c = threadIdx.x;
   float v[kChunks];
@@ -196,6 +199,11 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
   const int bh = blockIdx.y;
   const int which = blockIdx.z;
   const int b = bh / p.H, h = bh % p.H;
+  // Launched as a dependent of the K-mean combine: Q blocks start at once (they
+  // read only the inputs, written before the K-mean pass began), K blocks need the
+  // mean and V blocks the cleared V scale maximum, so they wait for the combine
+  // (which itself waited for the K-mean pass) to complete.
+  if (which != 0) pdl_wait();
   const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
   const int n_base = blk * 128;
   const int nq = (p.N + 127) / 128, nk = (p.N + 63) / 64;
@@ -234,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
   if (which == 0) {
     quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr,
                   INT8);
+    pdl_trigger();  // the attention kernel may be scheduled
     return;
   }
   if (which == 1) {
@@ -249,11 +258,13 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
     float* s1 = (2 * blk + 1 < nk) ? p.k_scale + bh * nk + 2 * blk + 1 : &unused_scale;
     quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr,
                   INT8);
+    pdl_trigger();
     return;
   }
   float* s1 = (2 * blk + 1 < nk) ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
   quantize_tile(x, true, n_base, p.N, p.v8 + out_off, cc, tl, red, p.v_scale + bh * nk + 2 * blk, s1,
                 p.v_scale_max + bh);
+  pdl_trigger();
 }
 
 }  // namespace
@@ -264,15 +275,11 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
   kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  kmean_finalize<<<p.B * p.H, 128, 0, stream>>>(p, partial);
-  e = cudaGetLastError();
+  e = launch_dependent(kmean_finalize, dim3(p.B * p.H), dim3(128), 0, stream, p, static_cast<const float*>(partial));
   if (e != cudaSuccess) return e;
   dim3 g2((p.N + 127) / 128, p.B * p.H, 3);
-  if (p.qk_int8)
-    quantize_qkv<true><<<g2, kThreads, 0, stream>>>(p);
-  else
-    quantize_qkv<false><<<g2, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return p.qk_int8 ? launch_dependent(quantize_qkv<true>, g2, dim3(kThreads), 0, stream, p)
+                   : launch_dependent(quantize_qkv<false>, g2, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace dit

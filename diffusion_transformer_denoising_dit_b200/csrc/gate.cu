@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_pass1(const __nv_bfloat16* 
                                                            const __nv_bfloat16* __restrict__ b, int64_t n,
                                                            double* __restrict__ partials) {
   // the dependent combine may be scheduled now; it waits for this grid to complete
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_trigger();
   float num = 0.f, den = 0.f;
   const int64_t n8 = n / 8;
   const uint4* a8 = reinterpret_cast<const uint4*>(a);
@@ -157,7 +157,7 @@ __device__ __forceinline__ void decide(double num, double den, float threshold, 
 __global__ void __launch_bounds__(kCombineThreads) gate_pass2(const double* __restrict__ partials, int nparts,
                                                               float threshold, float* __restrict__ rel_out,
                                                               int32_t* __restrict__ skip_out) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   double tn, td;
   combine_partials(partials, nparts, tn, td);
   if (threadIdx.x == 0) decide(tn, td, threshold, rel_out, skip_out);
@@ -167,30 +167,13 @@ __global__ void __launch_bounds__(kCombineThreads) gate_pass2(const double* __re
 // across ranks before gate_finalize decides.
 __global__ void __launch_bounds__(kCombineThreads) gate_pass2_sums(const double* __restrict__ partials, int nparts,
                                                                    double* __restrict__ sums_out) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   double tn, td;
   combine_partials(partials, nparts, tn, td);
   if (threadIdx.x == 0) {
     sums_out[0] = tn;
     sums_out[1] = td;
   }
-}
-
-// Launches a one-CTA combine as a programmatic dependent of the kernel before it
-// on the stream.
-template <typename... Params, typename... Args>
-cudaError_t launch_dependent(void (*kernel)(Params...), cudaStream_t stream, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
-  cfg.blockDim = dim3(kCombineThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 __global__ void gate_finalize(const double* __restrict__ sums, float threshold, float* __restrict__ rel_out,
@@ -205,7 +188,8 @@ cudaError_t launch_gate(const void* a, const void* b, int64_t n, float threshold
                                              static_cast<const __nv_bfloat16*>(b), n, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_dependent(gate_pass2, stream, static_cast<const double*>(partials), g, threshold, rel_out, skip_out);
+  return launch_dependent(gate_pass2, dim3(1), dim3(kCombineThreads), 0, stream, static_cast<const double*>(partials), g,
+                          threshold, rel_out, skip_out);
 }
 
 cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* sums_out, double* partials,
@@ -215,7 +199,8 @@ cudaError_t launch_gate_sums(const void* a, const void* b, int64_t n, double* su
                                              static_cast<const __nv_bfloat16*>(b), n, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_dependent(gate_pass2_sums, stream, static_cast<const double*>(partials), g, sums_out);
+  return launch_dependent(gate_pass2_sums, dim3(1), dim3(kCombineThreads), 0, stream,
+                          static_cast<const double*>(partials), g, sums_out);
 }
 
 cudaError_t launch_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
