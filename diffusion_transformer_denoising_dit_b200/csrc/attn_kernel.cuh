@@ -265,10 +265,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int NK = C::NK, NV = C::NV, BM = C::BM, BN = C::BN;
   // device-side skip (the cache gate's flag): the whole CTA leaves before any
   // barrier, TMEM allocation or load, so an early return is safe
-  if (out.skip != nullptr) {
-    pdl_wait();  // the flag's writer is visible once the kernel before this one has completed
-    if (*out.skip != 0) return;
-  }
+  if (out.skip != nullptr && *out.skip != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // Q0, Q1
@@ -346,10 +343,9 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Launched as a programmatic dependent of the kernel before it (FP8: the
-  // prologue's quantiser; BF16: the K rotation pass, when there is one):
-  // everything above may overlap that kernel's last CTAs, and nothing below reads
-  // its outputs before this wait
+  // FP8 is launched as a programmatic dependent of its prologue's quantiser:
+  // everything above may overlap the quantiser's last CTAs, and nothing below reads
+  // its outputs before this wait (a no-op for BF16's plain launch)
   pdl_wait();
 
   if (warp >= 8) {
@@ -942,9 +938,13 @@ cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
       cudaFuncSetAttribute(attn_kernel<FP8, D, I8QK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((out.N + 255) / 256, H, B);
-  // a programmatic dependent of the kernel before it on the stream (see pdl_wait in the kernel)
-  return launch_dependent(attn_kernel<FP8, D, I8QK>, grid, dim3(AttnCfg<FP8, D>::kThreads), smem, stream, tq, tk, tv,
-                          out, sc);
+  if constexpr (FP8)  // a programmatic dependent of the FP8 prologue's quantiser (see pdl_wait in the kernel)
+    return launch_dependent(attn_kernel<FP8, D, I8QK>, grid, dim3(AttnCfg<FP8, D>::kThreads), smem, stream, tq, tk,
+                            tv, out, sc);
+  // BF16: a plain launch (as a dependent of the K rotation pass it gained nothing
+  // measurable, and CUDA events around the call no longer bracketed its time)
+  attn_kernel<FP8, D, I8QK><<<grid, AttnCfg<FP8, D>::kThreads, smem, stream>>>(tq, tk, tv, out, sc);
+  return cudaGetLastError();
 }
 
 }  // namespace dit

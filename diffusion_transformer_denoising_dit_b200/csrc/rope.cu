@@ -117,7 +117,6 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
     rope8(*reinterpret_cast<const uint4*>(x + h * jb.sx[1]), cc, ss, y);
     store8(jb.y, yo + h * jb.sy[1], y, a.out_fp32);
   }
-  pdl_trigger();  // a dependent launch after this pass (the attention kernel) may be scheduled
 }
 
 cudaError_t launch_rope_apply(const RopeJob* jobs, int njobs, int B, int H, int N, int d, const float* cos_tab,
