@@ -52,12 +52,12 @@ FP8_GEMM_SUSTAINED_RECORDED = 2594.0
 # These are capture results, not measurements of this run; a kernel whose source
 # changed since its capture reports null.
 NCU_TRAFFIC = {
-    # attn_kernel<bf16, d=128>, 2048-px workload: 322.1 MB read + 86.3 MB written
-    ("attn_bf16", "87ce7b97f8480fae"): 408_391_424,
+    # attn_kernel<bf16, d=128>, 2048-px workload: 326.2 MB read + 86.4 MB written
+    ("attn_bf16", "d09989581d291e0f"): 412_548_352,
     # attn_kernel<fp8, d=128> (one hash covers both Q.K^T forms' source):
-    # e4m3 Q.K^T 155.8 + 71.7 MB; integer Q.K^T 156.9 + 71.0 MB
-    ("attn_fp8", "b8da0b2f5aea6883"): 227_558_400,
-    ("attn_fp8_i8qk", "b8da0b2f5aea6883"): 227_947_520,
+    # e4m3 Q.K^T 155.8 + 71.6 MB; integer Q.K^T 157.0 + 74.5 MB
+    ("attn_fp8", "f076ec4850baa389"): 227_420_160,
+    ("attn_fp8_i8qk", "f076ec4850baa389"): 231_572_224,
 }
 
 
