@@ -201,3 +201,32 @@ def test_fp8_smoothing_matters_for_shifted_keys(precision):
     model_gap = res[True][1] - res[False][1]
     assert model_gap > 0, res
     assert res[True][0] - res[False][0] >= 0.5 * model_gap, res
+
+
+def test_fp8_calls_on_two_streams_match_serial_calls():
+    """The FP8 call launches its prologue passes and the attention kernel as a chain
+    of programmatic dependent launches.  Calls of both variants running at the same
+    time on two streams (separate inputs and workspaces) give bit for bit what the
+    same calls give one after the other, and back-to-back calls on one stream that
+    reuse one workspace match them too."""
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=4)
+    cases = []
+    for seed, precision in ((11, "fp8"), (12, "fp8_i8qk")):
+        q, k, v, pos, cos, sin = _inputs(w, N=2048, seed=seed)
+        ws = dit.attention_workspace(*q.shape, precision=precision, device=DEV)
+        cases.append((q, k, v, cos, sin, precision, ws))
+    serial = []
+    for q, k, v, cos, sin, precision, ws in cases:
+        serial.append(dit.attention(q, k, v, cos, sin, precision=precision, workspace=ws).clone())
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in cases]
+    outs = []
+    torch.cuda.synchronize()
+    for (q, k, v, cos, sin, precision, ws), st in zip(cases, streams):
+        with torch.cuda.stream(st):
+            outs.append([dit.attention(q, k, v, cos, sin, precision=precision, workspace=ws) for _ in range(3)])
+    torch.cuda.synchronize()
+    assert dit.read_error() == 0
+    for ref, got in zip(serial, outs):
+        for o in got:
+            assert torch.equal(o, ref)
