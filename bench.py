@@ -324,6 +324,25 @@ def run_ours(args, rank, world, local_rank):
     def mcycles(ms, clk):
         return None if not clk.get("sm_mhz") else ms * clk["sm_mhz"] / 1e3
 
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    unit_rates = dit.probe_unit_rates()
+    ex2_rate = unit_rates["ex2_results"]
+    if not 4.0 <= ex2_rate <= 64.0:  # a probe reading outside any plausible SM: the B200 figure instead
+        ex2_rate = 16.0
+
+    def exp_roofline(ms, clk):
+        """The softmax's exponentials against the ex2 unit: B H N^2 exponentials per
+        call, against ex2.approx.f32 results per clock per SM as measured by the
+        unit-rate probe at the start of this run (16 on a B200; the packed f16x2 /
+        bf16x2 forms give no more results per clock), at the region's median clock."""
+        mhz = clk.get("sm_mhz") or 1965.0
+        exps = float(w.B * w.H * w.N * w.N)
+        achieved = exps / (ms / 1e3) / 1e9
+        peak = ex2_rate * n_sms * mhz * 1e6 / 1e9
+        return {"bound": "alu", "unit": "Gexp/s", "achieved": achieved, "peak": peak, "frac": achieved / peak,
+                "how": f"B H N^2 = {exps:.4g} exponentials per call / the call's time; peak = {ex2_rate:.2f} ex2 "
+                       f"per clock per SM (probed) x {n_sms} SMs x {mhz:.0f} MHz (the region's median clock)"}
+
     bf16_calls = [("attention", lambda: dit.attention(q, k, v, cos, sin, out=o, workspace=ws)),
                   ("gate", lambda: gate(r_cur, r_prev))]
 
@@ -354,7 +373,8 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_launch": ms_call,
                 "ms_per_launch_how": "mean over the timed steps of CUDA events around the attention call "
                                      "(K rotation pass + attention kernel) inside the headline region",
-                "sm_mcycles_per_launch": mcycles(ms_call, clocks)}
+                "sm_mcycles_per_launch": mcycles(ms_call, clocks),
+                "exp_roofline": exp_roofline(ms_call, clocks)}
 
     # ---- side kernels alone (HBM-bound): the K rotation pass and the gate
     kr2 = torch.empty_like(k)
@@ -408,6 +428,7 @@ def run_ours(args, rank, world, local_rank):
             "peak_nominal_ratio": fp8_peak, "frac_of_step_vs_2x_bf16": v8 / 1e12 / fp8_peak,
             "clocks": c8, "sm_mcycles_per_step": mcycles(mps8, c8),
             "step": f"{prec} call (prologue + attention) + fbcache_gate"}
+        fp8_objs[prec]["exp_roofline"] = exp_roofline(call8, c8)
         h8 = _src_hash("attn_kernel.cuh", "dit_device.cuh", "attn_fp8.cu")
         tr8 = NCU_TRAFFIC.get(("attn_fp8_i8qk" if prec == "fp8_i8qk" else "attn_fp8", h8))
         fp8_objs[prec]["attention_kernel_traffic"] = tr8
@@ -512,6 +533,7 @@ def run_ours(args, rank, world, local_rank):
             "fp8": fp8,
             "fp8_e4m3": fp8_e4m3,
             "side_kernels": side,
+            "unit_rates_per_clock_per_sm": unit_rates,
             "sm_mcycles_per_step": mcycles(ms_per_step, clocks),
             "accuracy": {
                 "bf16": "max-abs <= 2e-2 and cosine >= 0.9999 against exact attention on the bf16-rounded rotated "
@@ -763,6 +785,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--trace", action="store_true", help="run the 28-step denoising trace instead")
     ap.add_argument("--measure-fp8-peak", action="store_true", help="dense e4m3 GEMM peak (a denominator) instead")
+    ap.add_argument("--measure-unit-rates", action="store_true",
+                    help="tcgen05 MMA, ex2 and e4m3-conversion rates per clock per SM instead")
     ap.add_argument("--profile-attn", choices=["bf16", "fp8", "fp8_i8qk"],
                     help="a short fixed invocation for ncu captures instead of the benchmark")
     ap.add_argument("--profile-workload", default=WORKLOAD, choices=["flux1k", "flux2k"])
@@ -781,6 +805,22 @@ def main():
         return
     if args.measure_fp8_peak:
         run_fp8_peak()
+        return
+    if args.measure_unit_rates:
+        import torch
+        import diffusion_transformer_denoising_dit_b200 as dit
+        props = torch.cuda.get_device_properties(0)
+        r = dit.probe_unit_rates()
+        mhz = 1965.0
+        print(json.dumps({"per_clock_per_sm": r, "sms": props.multi_processor_count,
+                          "at_1965_mhz": {"mma_e4m3_TFLOP/s": r["mma_e4m3_flop"] * props.multi_processor_count
+                                          * mhz * 1e6 / 1e12,
+                                          "mma_bf16_TFLOP/s": r["mma_bf16_flop"] * props.multi_processor_count
+                                          * mhz * 1e6 / 1e12,
+                                          "ex2_Gexp/s": r["ex2_results"] * props.multi_processor_count * mhz / 1e3},
+                          "how": "dit_probe_unit_rates: device cycle counts of back-to-back tcgen05.mma "
+                                 "(M = N = 128, operands in shared memory), ex2.approx.f32 and "
+                                 "cvt.rn.satfinite.e4m3x2.f32"}), flush=True)
         return
     if args.profile_attn:
         run_profile_case(args)

@@ -19,4 +19,5 @@ from ._binding import (  # noqa: F401
     rope_apply,
     rope_tables,
     selftest_wait_timeout,
+    probe_unit_rates,
 )

@@ -22,7 +22,7 @@ EXPORTS = ["dit_status_string", "dit_read_error", "dit_rope_tables", "rope_apply
            "dit_attn_bf16_workspace_bytes", "dit_attn_bf16", "dit_attn_fp8_workspace_bytes",
            "dit_attn_fp8", "dit_attn_fp8_i8qk", "fbcache_gate_workspace_bytes", "fbcache_gate", "fbcache_gate_noalloc",
            "dit_selftest_wait_timeout", "dit_attn_bf16_skippable", "fbcache_gate_sums", "fbcache_gate_finalize",
-           "fbcache_gate_ref_update"]
+           "fbcache_gate_ref_update", "dit_probe_unit_rates"]
 
 
 class DitError(RuntimeError):
@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.dit_read_error.argtypes = [_vp]
         L.dit_selftest_wait_timeout.restype = _i
         L.dit_selftest_wait_timeout.argtypes = [_vp]
+        L.dit_probe_unit_rates.restype = _i
+        L.dit_probe_unit_rates.argtypes = [_vp, _i, _vp]
         L.dit_rope_tables.restype = _i
         L.dit_rope_tables.argtypes = [_vp, _i, _i, _i, _i, ctypes.c_double, _vp, _vp, _vp]
         L.rope_apply.restype = _i
@@ -152,6 +154,16 @@ def selftest_wait_timeout(stream=None) -> None:
     (read it with read_error())."""
     s = torch.cuda.current_stream().cuda_stream if stream is None else stream
     _check("dit_selftest_wait_timeout", lib().dit_selftest_wait_timeout(s))
+
+
+def probe_unit_rates(stream=None) -> dict:
+    """The hardware rates the kernels' rooflines are drawn against, per clock per
+    SM, measured on the current device (see dit_probe_unit_rates)."""
+    import ctypes
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    out = (ctypes.c_double * 4)()
+    _check("dit_probe_unit_rates", lib().dit_probe_unit_rates(ctypes.cast(out, ctypes.c_void_p), 4, s))
+    return {"mma_e4m3_flop": out[0], "mma_bf16_flop": out[1], "ex2_results": out[2], "cvt_e4m3x2_instructions": out[3]}
 
 
 def rope_tables(pos: torch.Tensor, axes, theta: float = 10000.0):

@@ -21,7 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdit.so")
 LIB_DEBUG = os.path.join(PKG, "libdit_debug.so")
-SOURCES = ["capi.cu", "rope.cu", "gate.cu", "attn_bf16.cu", "attn_fp8.cu", "fp8_prologue.cu", "selftest.cu"]
+SOURCES = ["capi.cu", "rope.cu", "gate.cu", "attn_bf16.cu", "attn_fp8.cu", "fp8_prologue.cu", "selftest.cu",
+           "probe.cu"]
 HEADERS = ["dit_device.cuh", "dit_internal.h", "attn_kernel.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "--expt-relaxed-constexpr",

@@ -100,6 +100,21 @@ DIT_API dit_status dit_read_error(dit_stream_t stream);
  * DIT_ERR_TIMEOUT.  Returns DIT_ERR_UNSUPPORTED off sm_100. */
 DIT_API dit_status dit_selftest_wait_timeout(dit_stream_t stream);
 
+/* Unit-rate probes (no counterpart on the pages; they measure the hardware rates
+ * the attention kernels' rooflines are drawn against).  Runs four short probes
+ * on the current device, synchronously on `stream`, and writes per clock per SM
+ * (from device cycle counts, so independent of the clock they ran at):
+ *   out[0]  FLOP of tcgen05.mma kind::f8f6f4 (e4m3), M = 128, N = 128, both
+ *           operands in shared memory (the attention kernels' Q.K^T shape)
+ *   out[1]  FLOP of tcgen05.mma kind::f16 (bf16), same shape
+ *   out[2]  results of ex2.approx.f32 (the softmax's exponential)
+ *   out[3]  instructions of cvt.rn.satfinite.e4m3x2.f32 (two results each)
+ * n_out: capacity of out, at least 4.  Allocates and frees a few bytes of
+ * device memory.  Takes a few tens of milliseconds.  Returns DIT_ERR_INVALID_ARG
+ * for a null out or n_out < 4, DIT_ERR_UNSUPPORTED off sm_100, DIT_ERR_TIMEOUT if
+ * an MMA completion wait ran out, DIT_ERR_LAUNCH on a CUDA error. */
+DIT_API dit_status dit_probe_unit_rates(double* out, int n_out, dit_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Rotary embedding                                                          */
 /* ------------------------------------------------------------------------ */

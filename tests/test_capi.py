@@ -181,3 +181,15 @@ def test_no_gpu_means_unsupported_not_fallback():
     L = B.lib()
     assert _attn(L) == 2
     assert L.fbcache_gate(A16, A16, 100, 0.1, A16, A16, A16, 1 << 20, None) == 2
+
+
+def test_unit_rate_probe_argument_checks():
+    """dit_probe_unit_rates refuses a null output or too small a capacity before
+    touching a device; without a GPU it reports unsupported."""
+    L = B.lib()
+    buf = (ctypes.c_double * 4)()
+    assert L.dit_probe_unit_rates(None, 4, None) == 1
+    assert L.dit_probe_unit_rates(ctypes.cast(buf, ctypes.c_void_p), 3, None) == 1
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        assert L.dit_probe_unit_rates(ctypes.cast(buf, ctypes.c_void_p), 4, None) == 2
