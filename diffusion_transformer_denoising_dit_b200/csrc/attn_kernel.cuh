@@ -34,11 +34,12 @@
 // softmax has loaded it into registers.
 // The BF16 MMA thread issues, per key tile j:
 //     O0 += P0(j-1) V(j-1);  S0(j) = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1(j) = Q1 K(j)^T
-// The FP8 MMA thread issues, per key tile j:
-//     S0(j) (once softmax 0 has read S0(j-1));  S1(j) (likewise);
-//     O0 += P0(j-1) V(j-1);  O1 += P1(j-1) V(j-1)
-// and commits each PV to pv_done_i, which softmax i waits for before it
-// overwrites P_i or rescales O_i.  (The ordering argument below is BF16's.)
+// The FP8 MMA thread instead polls both warpgroups' hand-offs and issues
+// whatever is ready: S_i(j) once softmax i has read S_i(j-1) (s_free_i) and
+// K(j) has landed, O_i += P_i(j) V(j) once softmax i has stored P_i(j)
+// (p_ready_i) and V(j) has landed; it commits each PV to pv_done_i, which
+// softmax i waits for before it overwrites P_i or rescales O_i.  (The ordering
+// argument below is BF16's.)
 // tcgen05 MMAs from one thread are executed in issue order, so S_i(j) never
 // overwrites P_i(j-1) before PV_i(j-1) has read it, and a tcgen05.commit
 // tracks every MMA the thread issued before it: when softmax i sees S_i(j)
@@ -49,10 +50,11 @@
 // the two softmax warpgroups take turns on the ex2 unit (in FP8 they run
 // freely).  BF16 releases P_i(j) in two 64-key halves, so the MMA thread issues
 // the first half of PV_i(j) while the second half is still being
-// exponentiated.  Thread-to-thread hand-offs
-// (P ready -> MMA warp, the ping-pong turns) use named barriers, which are
-// far cheaper than an mbarrier round trip; mbarriers remain only where the
-// tensor core or the TMA unit signals.
+// exponentiated.  BF16's thread-to-thread hand-offs (P ready -> MMA warp, the
+// ping-pong turns) use named barriers, which are far cheaper than an mbarrier
+// round trip; FP8's (S free, P ready) are mbarriers, which the MMA lane can poll
+// side by side and which have a tile of slack; the tensor core and the TMA unit
+// signal through mbarriers in both.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -289,10 +291,11 @@ __global__ void __launch_bounds__(384, 1)
   //                 kBarPHalf + i   BF16: softmax i stored keys 0..63 of P (128 arrive, MMA warp syncs)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + C::kNumBars);
   // Raised by the first role whose bounded wait gives up; every other bounded
-  // wait then gives up too.  A role that gives up still performs the rest of its
-  // named-barrier schedule (arrivals and syncs, without the work between them),
-  // so a partner blocked on a named barrier is always released: named barriers
-  // cannot time out, and their schedule is balanced.
+  // wait then gives up too.  BF16: a role that gives up still performs the rest
+  // of its named-barrier schedule (arrivals and syncs, without the work between
+  // them), so a partner blocked on a named barrier is always released: named
+  // barriers cannot time out, and their schedule is balanced.  FP8 has no named
+  // barriers: every wait in it is bounded, so a role simply leaves.
   const uint32_t abort_flag = smem_u32(tmem_slot + 1);
   // Progress counters that pace the failure path (written on every path, read only
   // on the failure path): mma_done[i] = PReady_i generations the MMA warp has
