@@ -230,3 +230,31 @@ def test_fp8_calls_on_two_streams_match_serial_calls():
     for ref, got in zip(serial, outs):
         for o in got:
             assert torch.equal(o, ref)
+
+
+@pytest.mark.parametrize("precision", ["fp8", "fp8_i8qk"])
+@pytest.mark.parametrize("layout", ["bhnd", "bnhd"])
+def test_fp8_batched_ragged_and_strided(precision, layout):
+    """B = 2, H = 3, N = 700 (a ragged last tile and a last 128-token slab without
+    its second 64-token block), in the contiguous [B, H, N, d] layout and in the
+    strided [B, N, H, d] one: every row of every (b, h) against the model of the
+    kernel's arithmetic on its own codes, and against exact attention."""
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=3, outliers=False)
+    N = 700
+    q, k, v = synth.qkv(w, device=DEV, N=N, B=2, seed=31)
+    if layout == "bnhd":
+        q, k, v = (t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3) for t in (q, k, v))
+    pos = synth.positions(w.T, int(math.isqrt(N - w.T)) + 1)[:N]
+    cos, sin = dit.rope_tables(pos.to(DEV), w.axes, w.theta)
+    ws = dit.attention_workspace(*q.shape, precision=precision, device=DEV)
+    o = dit.attention(q, k, v, cos, sin, precision=precision, workspace=ws)
+    assert dit.read_error() == 0
+    rows = np.arange(N)
+    exact = A.attention(q.cpu(), k.cpu(), v.cpu(), pos=pos.numpy(), axes=w.axes, theta=w.theta)
+    mod = _model_on_kernel_codes(ws, q.shape, precision, rows)
+    o = o.cpu().double().numpy()
+    assert _cos(o, mod) >= MODEL_COS, _cos(o, mod)
+    assert _cos(o, exact) >= TARGET_COS, _cos(o, exact)
+    for b in range(2):  # no (b, h) may be off on its own
+        for h in range(3):
+            assert _cos(o[b, h], mod[b, h]) >= MODEL_COS, (b, h, _cos(o[b, h], mod[b, h]))
