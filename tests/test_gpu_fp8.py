@@ -66,7 +66,7 @@ def _warps(N, picks):
     return np.concatenate([np.arange(s0, min(s0 + 32, N)) for s0 in starts])
 
 
-def _model_on_kernel_codes(ws, shape, precision, rows):
+def _model_on_kernel_codes(ws, shape, precision, rows, scale=None):
     """The arithmetic model run on the codes and block scales the prologue wrote."""
     B, H, N, d = shape
     vw = dit.fp8_workspace_views(ws, B, H, N, d)
@@ -75,7 +75,8 @@ def _model_on_kernel_codes(ws, shape, precision, rows):
     k8 = vw["k8"].cpu().view(qk_t).double().numpy()
     v8 = vw["v8"].cpu().view(torch.float8_e4m3fn).double().numpy()
     sc = {n: vw[n].cpu().double().numpy() for n in ("q_scale", "k_scale", "v_scale")}
-    return kernel_model_codes(q8, k8, v8, sc["q_scale"], sc["k_scale"], sc["v_scale"], rows, qk=QK[precision])
+    return kernel_model_codes(q8, k8, v8, sc["q_scale"], sc["k_scale"], sc["v_scale"], rows, scale=scale,
+                              qk=QK[precision])
 
 
 def _run(w, precision, N=None, seed=None, rows=None, smooth=True):
@@ -258,3 +259,21 @@ def test_fp8_batched_ragged_and_strided(precision, layout):
     for b in range(2):  # no (b, h) may be off on its own
         for h in range(3):
             assert _cos(o[b, h], mod[b, h]) >= MODEL_COS, (b, h, _cos(o[b, h], mod[b, h]))
+
+
+@pytest.mark.parametrize("precision", ["fp8", "fp8_i8qk"])
+def test_fp8_explicit_softmax_scale(precision):
+    """An explicit softmax scale (0.05 instead of 1/sqrt(d)) reaches both the
+    kernel and its model: the call tracks the model run with that scale and exact
+    attention with it."""
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2, outliers=False)
+    q, k, v, pos, cos, sin = _inputs(w, N=700, seed=41)
+    ws = dit.attention_workspace(*q.shape, precision=precision, device=DEV)
+    o = dit.attention(q, k, v, cos, sin, precision=precision, workspace=ws, scale=0.05)
+    assert dit.read_error() == 0
+    rows = np.arange(q.shape[2])
+    exact = A.attention(q.cpu(), k.cpu(), v.cpu(), scale=0.05, pos=pos, axes=w.axes, theta=w.theta)
+    mod = _model_on_kernel_codes(ws, q.shape, precision, rows, scale=0.05)
+    o = o.cpu().double().numpy()
+    assert _cos(o, mod) >= MODEL_COS, _cos(o, mod)
+    assert _cos(o, exact) >= TARGET_COS, _cos(o, exact)
