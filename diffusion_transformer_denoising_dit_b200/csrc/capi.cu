@@ -23,6 +23,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   bool probed = false;
   bool sm100 = false;
+  int sms = 0;         // multiprocessor count
   int* err = nullptr;  // device address of g_dit_error_word
 };
 
@@ -41,6 +42,8 @@ const DeviceState* device_state() {
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     s.sm100 = (major == 10 && minor == 0);
+    cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (s.sms < 1) s.sm100 = false;
     void* p = nullptr;
     if (s.sm100 && cudaGetSymbolAddress(&p, g_dit_error_word) == cudaSuccess) s.err = static_cast<int*>(p);
     if (!s.err) s.sm100 = false;
@@ -317,6 +320,8 @@ dit_status attn_fp8_impl(const void* q, const void* k, const void* v, void* o, i
   p.k_mean = reinterpret_cast<float*>(w); w += align256(bh * d * 4);
   p.v_scale_max = reinterpret_cast<float*>(w); w += align256(bh * 4);
   p.k_partial = reinterpret_cast<float*>(w);
+  p.err = ds->err;
+  p.num_sms = ds->sms;
 
   const int64_t cs[3] = {static_cast<int64_t>(H) * N * d, static_cast<int64_t>(N) * d, d};
   // Every map is built before the first launch, so an error return leaves nothing enqueued.

@@ -111,6 +111,8 @@ struct Fp8Prep {
   float* k_mean;    // [B*H][d]
   float* v_scale_max;  // [B*H]
   float* k_partial;    // [B*H][kFp8MeanChunks][128] K-mean partial sums
+  int* err;            // device error word (a staged copy that timed out)
+  int num_sms;         // the quantiser runs one persistent CTA per SM
 };
 
 constexpr int kFp8MeanChunks = 48;

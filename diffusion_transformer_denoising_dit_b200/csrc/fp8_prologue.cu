@@ -63,18 +63,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float m = red[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-  return m;
-}
-
 __global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __restrict__ partial) {
   pdl_trigger();  // the mean's combine (and through it the quantiser) may be scheduled
   const int bh = blockIdx.y;
@@ -87,11 +75,24 @@ __global__ void __launch_bounds__(kThreads) kmean_partial(Fp8Prep p, float* __re
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (p.smooth_k) {
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
-    for (int n = n0 + tl; n < n1; n += 16) {
-      float y[8];
-      load_rotate8(kb + static_cast<int64_t>(n) * p.sk[2] + cc * 8, p.cos_tab, p.sin_tab, n, cc, p.d / 2, y);
+    // four tokens per step, all loads issued before the adds (tokens in the same
+    // order as one at a time)
+    for (int n = n0 + tl; n < n1; n += 64) {
+      float y[4][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += y[i];
+      for (int u = 0; u < 4; ++u) {
+        const int m = n + 16 * u;
+        if (m < n1)
+          load_rotate8(kb + static_cast<int64_t>(m) * p.sk[2] + cc * 8, p.cos_tab, p.sin_tab, m, cc, p.d / 2, y[u]);
+        else
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[u][i] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (n + 16 * u < n1) acc[i] += y[u][i];
     }
   }
   __shared__ float red[16][128 + 4];
@@ -122,149 +123,352 @@ __global__ void __launch_bounds__(128) kmean_finalize(Fp8Prep p, const float* __
   p.k_mean[bh * 128 + c] = p.smooth_k ? sum / static_cast<float>(p.N) : 0.f;
 }
 
-// Eight floats times inv (within [-127, 127]) -> eight int8 (two's complement),
-// rounded to nearest even, in token-row byte order.  fma(x, inv, 1.5 * 2^23)
-// rounds x * inv once to an integer (the float's unit in the last place is 1
-// there), and the float's low byte is then that integer modulo 256.
-__device__ __forceinline__ uint32_t s8_bits(float x, float inv) {
-  return __float_as_uint(__fmaf_rn(x, inv, 12582912.0f));
-}
-__device__ __forceinline__ uint32_t cvt_s8x4(const float* x, float inv) {
-  // byte_perm selector nibbles pick bytes of {y:x}: low bytes of the four codes, in order
-  const uint32_t ab = __byte_perm(s8_bits(x[0], inv), s8_bits(x[1], inv), 0x0040);
-  const uint32_t cd = __byte_perm(s8_bits(x[2], inv), s8_bits(x[3], inv), 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
-}
-__device__ __forceinline__ uint2 cvt_s8x8(const float (&x)[8], float inv) {
-  return make_uint2(cvt_s8x4(x, inv), cvt_s8x4(x + 4, inv));
+// ---------------------------------------------------------------------------
+// Pass 2: the quantiser, a persistent CTA per SM.  Work item = one 128-token
+// block of one (b,h): three tiles, Q, V and K, taken in that order; CTA c takes
+// items c, c + G, c + 2G, ... (G CTAs), so that the CTAs together stream
+// through the heads one after another.  Tiles and the rotary rows they need are
+// staged in shared memory by bulk copies issued ahead of use, so the reads
+// never wait on registers: three 32 KB tile slots (one per tensor; a slot is
+// refilled for the next item as soon as every thread has read it) and two
+// 64 KB table slots (cos and sin rows of 128 tokens, one per item in flight,
+// refilled two items ahead).  A producer warp issues the copies as slots are
+// released; sixteen warps convert a tile while the copies of the following
+// ones are in flight.
+//
+// Thread t owns channel chunk cc = t % 16 (channels 8cc .. 8cc+7) of tokens
+// t/16 + 32 i, i = 0..3, of the tile; for a tile of two 64-token blocks (K, V)
+// tokens i = 0, 1 lie in the first block and i = 2, 3 in the second.
+constexpr int kQzThreads = 512;              // converting threads
+constexpr int kQzBlock = kQzThreads + 32;     // + the producer warp
+constexpr int kTileBytes = 128 * 256;      // 128 tokens x 128 bf16 channels
+constexpr int kTabBytes = 2 * 128 * 256;   // cos then sin rows (64 fp32 each) of 128 tokens
+constexpr int kQzBarOff = 3 * kTileBytes + 2 * kTabBytes;
+constexpr int kQzSmem = kQzBarOff + 512;   // + 10 mbarriers, the abort flag, two halves of warp maxima
+static_assert(kQzSmem <= 227 * 1024, "the quantiser's staging exceeds a CTA's shared memory");
+
+enum QzKind { kQzQ = 0, kQzK = 1, kQzV = 2 };
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
-// Quantises one 128-token block of one tensor held as 8 chunks per thread:
-// thread t owns channel chunk (t % 16) of tokens t/16 + 16 i, i = 0..7.  With
-// two_blocks the first four tokens of a thread lie in the first 64-token block.
-// int8: symmetric int8 codes and scales amax/127 instead of e4m3 and amax/448.
-__device__ __forceinline__ void quantize_tile(float (&x)[8][8], bool two_blocks, int n_base, int N,
-                                              uint8_t* __restrict__ dst, int cc, int tl, float* red, float* sc_out0,
-                                              float* sc_out1, float* vmax, bool int8 = false) {
+// One warp, all lanes: stage tokens [n0, n0 + rows) of one (b,h) slab of a bf16
+// tensor (token stride ts elements; a token's 128 channels contiguous and
+// 16-byte aligned) into a tile slot, 256 bytes per token.
+__device__ __forceinline__ void stage_tile(uint8_t* slot, uint64_t* bar, const __nv_bfloat16* slab, int64_t ts,
+                                           int n0, int rows) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * 256u);
+  __syncwarp();
+  if (ts == 128) {
+    if (lane == 0) bulk_g2s(slot, slab + static_cast<int64_t>(n0) * 128, static_cast<uint32_t>(rows) * 256u, bar);
+  } else {
+    for (int r = lane; r < rows; r += 32) bulk_g2s(slot + r * 256, slab + static_cast<int64_t>(n0 + r) * ts, 256u, bar);
+  }
+}
+
+// One warp: stage the cos and sin rows of tokens [n0, n0 + rows) into a table slot.
+__device__ __forceinline__ void stage_tables(uint8_t* slot, uint64_t* bar, const float* cos_tab, const float* sin_tab,
+                                             int n0, int rows) {
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t bytes = static_cast<uint32_t>(rows) * 256u;
+    mbar_arrive_expect_tx(bar, 2u * bytes);
+    bulk_g2s(slot, cos_tab + static_cast<int64_t>(n0) * 64, bytes, bar);
+    bulk_g2s(slot + kTabBytes / 2, sin_tab + static_cast<int64_t>(n0) * 64, bytes, bar);
+  }
+  __syncwarp();
+}
+
+// Named barrier 1 over the 16 converting warps (the producer warp is not in it),
+// returning whether any of them passed true.
+__device__ __forceinline__ bool converters_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 512, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
+struct QzItem {
+  int bh, blk, n0, rows;
+};
+
+// item = bh * nq + blk
+__device__ __forceinline__ QzItem qz_item(const Fp8Prep& p, int item, int nq) {
+  QzItem r;
+  r.bh = item / nq;
+  r.blk = item - r.bh * nq;
+  r.n0 = r.blk * 128;
+  r.rows = min(128, p.N - r.n0);
+  return r;
+}
+
+__device__ __forceinline__ const __nv_bfloat16* qz_slab(const Fp8Prep& p, int kind, int bh) {
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const void* base = kind == kQzQ ? p.q : kind == kQzK ? p.k : p.v;
+  const int64_t* s = kind == kQzQ ? p.sq : kind == kQzK ? p.sk : p.sv;
+  return static_cast<const __nv_bfloat16*>(base) + b * s[0] + h * s[1];
+}
+
+__device__ __forceinline__ int64_t qz_stride(const Fp8Prep& p, int kind) {
+  return kind == kQzQ ? p.sq[2] : kind == kQzK ? p.sk[2] : p.sv[2];
+}
+
+// One tile: read the staged rows, rotate (Q, K), subtract the K mean, block
+// maxima, then scale, cast and store.  Returns false when a staged copy did not
+// arrive in time or the producer gave up (uniform over the converting warps).
+// Each warp releases the tile slot (and, for K, the table slot: K is the last
+// reader of an item's rows) with one arrival as soon as its reads are done.
+// red: this tile's half of the double-buffered warp maxima (two consecutive
+// tiles never share a half, so one barrier per tile suffices).
+//
+// A token's eight channels are held as four fp32 pairs (sm_100 f32x2
+// arithmetic): ev[q] = channels (4q, 4q + 2), od[q] = (4q + 1, 4q + 3), so that
+// the rotary pairs (2j, 2j + 1), j = 2q, 2q + 1, sit in matching lanes of ev and
+// od, and the tables' cos and sin (j, j + 1) load as one pair each.
+template <int KIND, bool INT8>
+__device__ __forceinline__ bool qz_tile(const Fp8Prep& p, const QzItem& it, const uint8_t* tile, uint64_t* tile_bar,
+                                        uint64_t* tile_empty, uint32_t tile_par, const uint8_t* tab,
+                                        uint64_t* tab_bar, uint64_t* tab_empty, uint32_t tab_par, float* red,
+                                        uint32_t abort_flag) {
+  const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool rot = KIND != kQzV && p.cos_tab != nullptr;
+  uint64_t nmean[4];  // K: minus the channel means, in the ev / od lane order
+  if (KIND == kQzK) {
+    const float4 m0 = *reinterpret_cast<const float4*>(p.k_mean + it.bh * 128 + cc * 8);
+    const float4 m1 = *reinterpret_cast<const float4*>(p.k_mean + it.bh * 128 + cc * 8 + 4);
+    nmean[0] = f2(-m0.x, -m0.z);
+    nmean[1] = f2(-m0.y, -m0.w);
+    nmean[2] = f2(-m1.x, -m1.z);
+    nmean[3] = f2(-m1.y, -m1.w);
+  }
+  bool ok = mbar_wait(tile_bar, tile_par, p.err, kErrTimeout, abort_flag);
+  if (rot) ok = ok && mbar_wait(tab_bar, tab_par, p.err, kErrTimeout, abort_flag);
+  const uint64_t minus1 = f2(-1.f, -1.f);
+  uint64_t ev[4][2], od[4][2];
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < 4; ++i) {
+    const int t = tl + 32 * i;
+    if (ok && t < it.rows) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(tile + t * 256 + cc * 16);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};  // bf16 pairs, low half = even channel
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (i < 4 || !two_blocks)
-        a0 = fmaxf(a0, fabsf(x[i][e]));
-      else
-        a1 = fmaxf(a1, fabsf(x[i][e]));
-    }
-  a0 = block_max(a0, red);
-  if (two_blocks) a1 = block_max(a1, red + 8);
-  const float qmax = int8 ? 127.f : 448.f;
-  const float s0 = a0 > 0.f ? a0 / qmax : 1.f;
-  const float s1 = a1 > 0.f ? a1 / qmax : 1.f;
-  const float inv0 = a0 > 0.f ? qmax / a0 : 1.f;
-  const float inv1 = a1 > 0.f ? qmax / a1 : 1.f;
-  if (threadIdx.x == 0) {
-    *sc_out0 = s0;
-    if (two_blocks) *sc_out1 = s1;
-    if (vmax) {
-      atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s0));
-      // a second block past the sequence end (all zeros, scale 1) is not a V block
-      if (two_blocks && n_base + 64 < N) atomicMax(reinterpret_cast<int*>(vmax), __float_as_int(s1));
-    }
-  }
+      for (int q = 0; q < 2; ++q) {
+        ev[i][q] = f2(__uint_as_float(w[2 * q] << 16), __uint_as_float(w[2 * q + 1] << 16));
+        od[i][q] = f2(__uint_as_float(w[2 * q] & 0xffff0000u), __uint_as_float(w[2 * q + 1] & 0xffff0000u));
+      }
+      if (rot) {
+        const uint4 c = *reinterpret_cast<const uint4*>(tab + t * 256 + cc * 16);
+        const uint4 s = *reinterpret_cast<const uint4*>(tab + kTabBytes / 2 + t * 256 + cc * 16);
+        const uint64_t c2[2] = {f2(__uint_as_float(c.x), __uint_as_float(c.y)),
+                                f2(__uint_as_float(c.z), __uint_as_float(c.w))};
+        const uint64_t s2[2] = {f2(__uint_as_float(s.x), __uint_as_float(s.y)),
+                                f2(__uint_as_float(s.z), __uint_as_float(s.w))};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = n_base + tl + 16 * i;
-    if (n >= N) continue;
-    const float inv = (i < 4 || !two_blocks) ? inv0 : inv1;
-    uint2 w;
-    if (int8) {
-      w = cvt_s8x8(x[i], inv);
+        for (int q = 0; q < 2; ++q) {
+          // (x_e, x_o) -> (x_e c - x_o s, x_e s + x_o c)
+          const uint64_t e = ev[i][q], o = od[i][q];
+          ev[i][q] = ffma2(o, fmul2(s2[q], minus1), fmul2(e, c2[q]));
+          od[i][q] = ffma2(o, c2[q], fmul2(e, s2[q]));
+        }
+      }
+      if (KIND == kQzK) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          ev[i][q] = fadd2(ev[i][q], nmean[2 * q]);
+          od[i][q] = fadd2(od[i][q], nmean[2 * q + 1]);
+        }
+      }
     } else {
-      w.x = cvt_e4m3x2(x[i][0] * inv, x[i][1] * inv) | (cvt_e4m3x2(x[i][2] * inv, x[i][3] * inv) << 16);
-      w.y = cvt_e4m3x2(x[i][4] * inv, x[i][5] * inv) | (cvt_e4m3x2(x[i][6] * inv, x[i][7] * inv) << 16);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) ev[i][q] = od[i][q] = 0ull;
     }
-    *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(n) * 128 + cc * 8) = w;
-  }
-}
-
-// One CTA per (128-token block, (b,h), tensor): blockIdx.z = 0 quantises Q (one
-// 128-token block, rotated), 1 quantises K (two 64-token blocks, rotated and
-// smoothed), 2 quantises V (two 64-token blocks).  Every thread issues its eight
-// 16-byte loads before any reduction, so each CTA keeps 32 KB in flight.
-// INT8: Q and K as symmetric int8 (the integer Q.K^T form), V as e4m3.
-template <bool INT8>
-__global__ void __launch_bounds__(kThreads, 3) quantize_qkv(Fp8Prep p) {
-  const int blk = blockIdx.x;  // 128-token block
-  const int bh = blockIdx.y;
-  const int which = blockIdx.z;
-  const int b = bh / p.H, h = bh % p.H;
-  // Launched as a dependent of the K-mean combine: Q blocks start at once (they
-  // read only the inputs, written before the K-mean pass began), K blocks need the
-  // mean and V blocks the cleared V scale maximum, so they wait for the combine
-  // (which itself waited for the K-mean pass) to complete.
-  if (which != 0) pdl_wait();
-  const int cc = threadIdx.x & 15, tl = threadIdx.x >> 4;
-  const int n_base = blk * 128;
-  const int nq = (p.N + 127) / 128, nk = (p.N + 63) / 64;
-  __shared__ float mean[128];
-  __shared__ float red[16];
-  __shared__ float unused_scale;  // sink for the second scale of a block past the sequence end
-  const int64_t out_off = static_cast<int64_t>(bh) * p.N * 128;
-  const __nv_bfloat16* src;
-  int64_t tok_stride;
-  const float* ct = nullptr;
-  const float* st = nullptr;
-  if (which == 0) {
-    src = static_cast<const __nv_bfloat16*>(p.q) + b * p.sq[0] + h * p.sq[1];
-    tok_stride = p.sq[2];
-    ct = p.cos_tab;
-    st = p.sin_tab;
-  } else if (which == 1) {
-    src = static_cast<const __nv_bfloat16*>(p.k) + b * p.sk[0] + h * p.sk[1];
-    tok_stride = p.sk[2];
-    ct = p.cos_tab;
-    st = p.sin_tab;
-  } else {
-    src = static_cast<const __nv_bfloat16*>(p.v) + b * p.sv[0] + h * p.sv[1];
-    tok_stride = p.sv[2];
-  }
-  float x[8][8];
+    float m = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = n_base + tl + 16 * i;
-    if (n < p.N)
-      load_rotate8(src + static_cast<int64_t>(n) * tok_stride + cc * 8, ct, st, n, cc, 64, x[i]);
+    for (int q = 0; q < 2; ++q) {
+      float e0, e1, o0, o1;
+      f2_split(ev[i][q], e0, e1);
+      f2_split(od[i][q], o0, o1);
+      m = fmax3(m, fabsf(e0), fabsf(e1));
+      m = fmax3(m, fabsf(o0), fabsf(o1));
+    }
+    if (KIND == kQzQ || i < 2)
+      a0 = fmaxf(a0, m);
     else
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+      a1 = fmaxf(a1, m);
   }
-  if (which == 0) {
-    quantize_tile(x, false, n_base, p.N, p.q8 + out_off, cc, tl, red, p.q_scale + bh * nq + blk, nullptr, nullptr,
-                  INT8);
-    pdl_trigger();  // the attention kernel may be scheduled
-    return;
+  __syncwarp();  // the warp's reads of the slots are done
+  if (lane == 0) {
+    mbar_arrive(tile_empty);
+    if (KIND == kQzK && rot) mbar_arrive(tab_empty);
   }
-  if (which == 1) {
-    if (threadIdx.x < 128) mean[threadIdx.x] = p.k_mean[bh * 128 + threadIdx.x];
-    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (n_base + tl + 16 * i < p.N) {
+  for (int o = 16; o > 0; o >>= 1) {
+    a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, o));
+    if (KIND != kQzQ) a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, o));
+  }
+  if (lane == 0) {
+    red[warp] = a0;
+    red[16 + warp] = a1;
+  }
+  // every warp's maxima are in red
+  if (converters_sync_or(!ok)) return false;
+  float m = red[lane];  // lanes 0-15: first block, 16-31: second
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] -= mean[cc * 8 + e];
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float b0 = __shfl_sync(0xffffffffu, m, 0), b1 = __shfl_sync(0xffffffffu, m, 16);
+  const float qmax = (INT8 && KIND != kQzV) ? 127.f : 448.f;
+  const float inv0 = b0 > 0.f ? qmax / b0 : 1.f;
+  const float inv1 = (KIND != kQzQ && b1 > 0.f) ? qmax / b1 : 1.f;
+  if (threadIdx.x == 0) {
+    const float s0 = b0 > 0.f ? b0 / qmax : 1.f, s1 = b1 > 0.f ? b1 / qmax : 1.f;
+    const int nq = (p.N + 127) / 128, nk = (p.N + 63) / 64;
+    if (KIND == kQzQ) {
+      p.q_scale[it.bh * nq + it.blk] = s0;
+    } else {
+      float* sc = (KIND == kQzK ? p.k_scale : p.v_scale) + it.bh * nk + 2 * it.blk;
+      sc[0] = s0;
+      const bool second = 2 * it.blk + 1 < nk;  // a second 64-token block inside the sequence
+      if (second) sc[1] = s1;
+      if (KIND == kQzV) {
+        atomicMax(reinterpret_cast<int*>(p.v_scale_max + it.bh), __float_as_int(s0));
+        if (second) atomicMax(reinterpret_cast<int*>(p.v_scale_max + it.bh), __float_as_int(s1));
       }
     }
-    float* s1 = (2 * blk + 1 < nk) ? p.k_scale + bh * nk + 2 * blk + 1 : &unused_scale;
-    quantize_tile(x, true, n_base, p.N, p.k8 + out_off, cc, tl, red, p.k_scale + bh * nk + 2 * blk, s1, nullptr,
-                  INT8);
-    pdl_trigger();
+  }
+  uint8_t* dst = (KIND == kQzQ ? p.q8 : KIND == kQzK ? p.k8 : p.v8) + static_cast<int64_t>(it.bh) * p.N * 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = tl + 32 * i;
+    if (t >= it.rows) continue;
+    const float inv = (KIND == kQzQ || i < 2) ? inv0 : inv1;
+    uint32_t wd[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float e0, e1, o0, o1;  // channels 4q, 4q + 2 and 4q + 1, 4q + 3
+      if (INT8 && KIND != kQzV) {
+        // int8 codes: fma(x, inv, 1.5 * 2^23) rounds x * inv (within [-127, 127]) once
+        // to the nearest integer, ties to even (the float's unit in the last place is 1
+        // there), and the float's low byte is then that integer modulo 256, i.e. its
+        // two's complement byte; byte permutes gather the four low bytes in channel order.
+        const uint64_t bias = f2(12582912.0f, 12582912.0f), inv2 = f2(inv, inv);
+        f2_split(ffma2(ev[i][q], inv2, bias), e0, e1);
+        f2_split(ffma2(od[i][q], inv2, bias), o0, o1);
+        const uint32_t lo = __byte_perm(__float_as_uint(e0), __float_as_uint(o0), 0x0040);
+        const uint32_t hi = __byte_perm(__float_as_uint(e1), __float_as_uint(o1), 0x0040);
+        wd[q] = __byte_perm(lo, hi, 0x5410);
+      } else {
+        const uint64_t inv2 = f2(inv, inv);
+        f2_split(fmul2(ev[i][q], inv2), e0, e1);
+        f2_split(fmul2(od[i][q], inv2), o0, o1);
+        wd[q] = cvt_e4m3x2(e0, o0) | (cvt_e4m3x2(e1, o1) << 16);
+      }
+    }
+    *reinterpret_cast<uint2*>(dst + static_cast<int64_t>(it.n0 + t) * 128 + cc * 8) = make_uint2(wd[0], wd[1]);
+  }
+  return true;
+}
+
+// INT8: Q and K as symmetric int8 (the integer Q.K^T form), V as e4m3.
+template <bool INT8>
+__global__ void __launch_bounds__(kQzBlock, 1) quantize_qkv(Fp8Prep p) {
+  extern __shared__ __align__(128) uint8_t qz_smem[];
+  uint8_t* tiles = qz_smem;                   // [3][kTileBytes]: slot = tensor (Q, K, V)
+  uint8_t* tabs = qz_smem + 3 * kTileBytes;  // [2][kTabBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qz_smem + kQzBarOff);
+  uint64_t* tile_full = bars;       // [3] one arrival (the producer's) + the copy's bytes
+  uint64_t* tab_full = bars + 3;    // [2]
+  uint64_t* tile_empty = bars + 5;  // [3] one arrival per converting warp
+  uint64_t* tab_empty = bars + 8;   // [2]
+  int* abort_flag = reinterpret_cast<int*>(bars + 10);
+  float* red = reinterpret_cast<float*>(qz_smem + kQzBarOff + 128);  // [2][32] warp maxima
+  // The attention kernel may be scheduled; it waits for this grid to complete.
+  pdl_trigger();
+  const int nq = (p.N + 127) / 128;
+  const int items = p.B * p.H * nq;
+  const int stride = gridDim.x;
+  const bool rope = p.cos_tab != nullptr;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+    for (int i = 5; i < 10; ++i) mbar_init(&bars[i], kQzThreads / 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint32_t abort_a = smem_u32(abort_flag);
+  if (threadIdx.x >= kQzThreads) {
+    // Producer warp: stages item n's rows (into table slot n % 2) and its Q, V and K
+    // tiles as soon as the slots' previous contents are released.
+    uint32_t staged = 0, last = 0;  // per full barrier (bit b): staged at all; parity of the last phase
+    bool ok = true;
+    int n = 0;
+    for (int item = blockIdx.x; item < items && ok; item += stride, ++n) {
+      const QzItem it = qz_item(p, item, nq);
+      if (rope) {
+        const int ts = n & 1;
+        if (n >= 2) ok = mbar_wait(&tab_empty[ts], static_cast<uint32_t>((n - 2) >> 1) & 1u, p.err, kErrTimeout,
+                                   abort_a);
+        if (!ok) break;
+        stage_tables(tabs + ts * kTabBytes, &tab_full[ts], p.cos_tab, p.sin_tab, it.n0, it.rows);
+        staged |= 1u << (3 + ts);
+        last = (last & ~(1u << (3 + ts))) | ((static_cast<uint32_t>(n >> 1) & 1u) << (3 + ts));
+      }
+#pragma unroll
+      for (int j = 0; j < 3 && ok; ++j) {
+        const int kind = j == 0 ? kQzQ : j == 1 ? kQzV : kQzK;
+        if (n >= 1) ok = mbar_wait(&tile_empty[kind], static_cast<uint32_t>(n - 1) & 1u, p.err, kErrTimeout, abort_a);
+        if (!ok) break;
+        stage_tile(tiles + kind * kTileBytes, &tile_full[kind], qz_slab(p, kind, it.bh), qz_stride(p, kind), it.n0,
+                   it.rows);
+        staged |= 1u << kind;
+        last = (last & ~(1u << kind)) | ((static_cast<uint32_t>(n) & 1u) << kind);
+      }
+    }
+    if (!ok && (threadIdx.x & 31) == 0) {
+      // The converting warps stopped (or a release timed out, recorded in the error
+      // word): wait, bounded, for every copy staged before the CTA's shared memory
+      // is released.
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+#pragma unroll
+      for (int b = 0; b < 5; ++b)
+        if ((staged >> b) & 1u) mbar_wait_until(&bars[b], (last >> b) & 1u, deadline);
+    }
     return;
   }
-  float* s1 = (2 * blk + 1 < nk) ? p.v_scale + bh * nk + 2 * blk + 1 : &unused_scale;
-  quantize_tile(x, true, n_base, p.N, p.v8 + out_off, cc, tl, red, p.v_scale + bh * nk + 2 * blk, s1,
-                p.v_scale_max + bh);
-  pdl_trigger();
+  int n = 0;
+  for (int item = blockIdx.x; item < items; item += stride, ++n) {
+    const QzItem it = qz_item(p, item, nq);
+    const int ts = n & 1;
+    const uint32_t tpar = static_cast<uint32_t>(n) & 1u, bpar = static_cast<uint32_t>(n >> 1) & 1u;
+    // warp-maxima halves alternate tile by tile (Q, V, K, Q, ...: 3n, 3n + 1, 3n + 2)
+    float* red_a = red + 32 * (n & 1);
+    float* red_b = red + 32 * ((n + 1) & 1);
+    uint8_t* tab = tabs + ts * kTabBytes;
+    // Q: reads only the inputs, written before the K-mean pass began.
+    bool ok = qz_tile<kQzQ, INT8>(p, it, tiles + kQzQ * kTileBytes, &tile_full[kQzQ], &tile_empty[kQzQ], tpar, tab,
+                                  &tab_full[ts], &tab_empty[ts], bpar, red_a, abort_a);
+    // V needs the cleared per-(b,h) scale maximum and K the channel means: both
+    // from the grids this one depends on.
+    if (ok && n == 0) pdl_wait();
+    ok = ok && qz_tile<kQzV, INT8>(p, it, tiles + kQzV * kTileBytes, &tile_full[kQzV], &tile_empty[kQzV], tpar,
+                                   nullptr, nullptr, nullptr, 0u, red_b, abort_a);
+    ok = ok && qz_tile<kQzK, INT8>(p, it, tiles + kQzK * kTileBytes, &tile_full[kQzK], &tile_empty[kQzK], tpar, tab,
+                                   &tab_full[ts], &tab_empty[ts], bpar, red_a, abort_a);
+    if (!ok) {
+      if (threadIdx.x == 0) flag_store(abort_a, 1);  // the producer stops and drains its copies
+      break;
+    }
+  }
 }
 
 }  // namespace
@@ -277,9 +481,13 @@ cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = launch_dependent(kmean_finalize, dim3(p.B * p.H), dim3(128), 0, stream, p, static_cast<const float*>(partial));
   if (e != cudaSuccess) return e;
-  dim3 g2((p.N + 127) / 128, p.B * p.H, 3);
-  return p.qk_int8 ? launch_dependent(quantize_qkv<true>, g2, dim3(kThreads), 0, stream, p)
-                   : launch_dependent(quantize_qkv<false>, g2, dim3(kThreads), 0, stream, p);
+  const int64_t items = static_cast<int64_t>(p.B) * p.H * ((p.N + 127) / 128);
+  if (items > 0x7fffffff || p.num_sms < 1) return cudaErrorInvalidValue;
+  const int grid = static_cast<int>(items < p.num_sms ? items : p.num_sms);  // persistent: one CTA per SM
+  auto kern = p.qk_int8 ? quantize_qkv<true> : quantize_qkv<false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQzSmem);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(kern, dim3(grid), dim3(kQzBlock), kQzSmem, stream, p);
 }
 
 }  // namespace dit
