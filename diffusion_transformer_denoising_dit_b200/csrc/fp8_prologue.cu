@@ -434,10 +434,12 @@ __global__ void __launch_bounds__(kQzBlock, 1) quantize_qkv(Fp8Prep p) {
         last = (last & ~(1u << kind)) | ((static_cast<uint32_t>(n) & 1u) << kind);
       }
     }
-    if (!ok && (threadIdx.x & 31) == 0) {
-      // The converting warps stopped (or a release timed out, recorded in the error
-      // word): wait, bounded, for every copy staged before the CTA's shared memory
-      // is released.
+    if ((threadIdx.x & 31) == 0) {
+      // Wait, bounded, for every copy staged before the CTA's shared memory is
+      // released.  Needed on every exit, not only after a failed wait of this warp:
+      // the converting warps release their slots on their failure path too, which
+      // can let the last stagings through after they have stopped.  On the normal
+      // path the copies have landed or are about to (the converting warps wait for them).
       const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
 #pragma unroll
       for (int b = 0; b < 5; ++b)
