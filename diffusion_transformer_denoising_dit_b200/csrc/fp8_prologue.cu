@@ -158,26 +158,39 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // One warp, all lanes: stage tokens [n0, n0 + rows) of one (b,h) slab of a bf16
 // tensor (token stride ts elements; a token's 128 channels contiguous and
 // 16-byte aligned) into a tile slot, 256 bytes per token.
+// (Debug builds: a copy whose size or alignment fails its check is not issued;
+// its bytes never arrive, so the slot's wait times out after recording the error.)
 __device__ __forceinline__ void stage_tile(uint8_t* slot, uint64_t* bar, const __nv_bfloat16* slab, int64_t ts,
-                                           int n0, int rows) {
+                                           int n0, int rows, int* err) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * 256u);
   __syncwarp();
   if (ts == 128) {
-    if (lane == 0) bulk_g2s(slot, slab + static_cast<int64_t>(n0) * 128, static_cast<uint32_t>(rows) * 256u, bar);
+    const __nv_bfloat16* src = slab + static_cast<int64_t>(n0) * 128;
+    if (lane == 0 && debug_check(rows >= 1 && rows <= 128 && (reinterpret_cast<uintptr_t>(src) & 15) == 0, err))
+      bulk_g2s(slot, src, static_cast<uint32_t>(rows) * 256u, bar);
   } else {
-    for (int r = lane; r < rows; r += 32) bulk_g2s(slot + r * 256, slab + static_cast<int64_t>(n0 + r) * ts, 256u, bar);
+    for (int r = lane; r < rows; r += 32) {
+      const __nv_bfloat16* src = slab + static_cast<int64_t>(n0 + r) * ts;
+      if (debug_check(r < 128 && (reinterpret_cast<uintptr_t>(src) & 15) == 0, err))
+        bulk_g2s(slot + r * 256, src, 256u, bar);
+    }
   }
 }
 
 // One warp: stage the cos and sin rows of tokens [n0, n0 + rows) into a table slot.
 __device__ __forceinline__ void stage_tables(uint8_t* slot, uint64_t* bar, const float* cos_tab, const float* sin_tab,
-                                             int n0, int rows) {
+                                             int n0, int rows, int* err) {
   if ((threadIdx.x & 31) == 0) {
     const uint32_t bytes = static_cast<uint32_t>(rows) * 256u;
     mbar_arrive_expect_tx(bar, 2u * bytes);
-    bulk_g2s(slot, cos_tab + static_cast<int64_t>(n0) * 64, bytes, bar);
-    bulk_g2s(slot + kTabBytes / 2, sin_tab + static_cast<int64_t>(n0) * 64, bytes, bar);
+    const float* c = cos_tab + static_cast<int64_t>(n0) * 64;
+    const float* s = sin_tab + static_cast<int64_t>(n0) * 64;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(c) | reinterpret_cast<uintptr_t>(s);
+    if (debug_check(rows >= 1 && rows <= 128 && (a & 15) == 0, err)) {
+      bulk_g2s(slot, c, bytes, bar);
+      bulk_g2s(slot + kTabBytes / 2, s, bytes, bar);
+    }
   }
   __syncwarp();
 }
@@ -259,7 +272,7 @@ __device__ __forceinline__ bool qz_tile(const Fp8Prep& p, const QzItem& it, cons
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int t = tl + 32 * i;
-    if (ok && t < it.rows) {
+    if (ok && t < it.rows && debug_check(t < 128, p.err)) {
       const uint4 raw = *reinterpret_cast<const uint4*>(tile + t * 256 + cc * 16);
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};  // bf16 pairs, low half = even channel
 #pragma unroll
@@ -419,7 +432,7 @@ __global__ void __launch_bounds__(kQzBlock, 1) quantize_qkv(Fp8Prep p) {
         if (n >= 2) ok = mbar_wait(&tab_empty[ts], static_cast<uint32_t>((n - 2) >> 1) & 1u, p.err, kErrTimeout,
                                    abort_a);
         if (!ok) break;
-        stage_tables(tabs + ts * kTabBytes, &tab_full[ts], p.cos_tab, p.sin_tab, it.n0, it.rows);
+        stage_tables(tabs + ts * kTabBytes, &tab_full[ts], p.cos_tab, p.sin_tab, it.n0, it.rows, p.err);
         staged |= 1u << (3 + ts);
         last = (last & ~(1u << (3 + ts))) | ((static_cast<uint32_t>(n >> 1) & 1u) << (3 + ts));
       }
@@ -429,7 +442,7 @@ __global__ void __launch_bounds__(kQzBlock, 1) quantize_qkv(Fp8Prep p) {
         if (n >= 1) ok = mbar_wait(&tile_empty[kind], static_cast<uint32_t>(n - 1) & 1u, p.err, kErrTimeout, abort_a);
         if (!ok) break;
         stage_tile(tiles + kind * kTileBytes, &tile_full[kind], qz_slab(p, kind, it.bh), qz_stride(p, kind), it.n0,
-                   it.rows);
+                   it.rows, p.err);
         staged |= 1u << kind;
         last = (last & ~(1u << kind)) | ((static_cast<uint32_t>(n) & 1u) << kind);
       }
