@@ -11,10 +11,24 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dit.h"
 #include "dit_internal.h"
 
 namespace {
+
+// One NVTX range per call, named after the entry point, around its host work and
+// launches: Nsight tools show it, and `ncu --nvtx --nvtx-include "<name>/"`
+// captures one call's kernels.  Without a tool attached a push and a pop cost a
+// few nanoseconds (NVTX v3, header only: a tool is loaded at the first call
+// from NVTX_INJECTION64_PATH, if set).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 __device__ int g_dit_error_word;
 
@@ -125,6 +139,7 @@ const char* dit_status_string(dit_status s) {
 }
 
 dit_status dit_read_error(dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_read_error");
   const DeviceState* ds = device_state();
   if (!ds || !ds->sm100) return DIT_ERR_UNSUPPORTED;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return DIT_ERR_LAUNCH;
@@ -136,6 +151,7 @@ dit_status dit_read_error(dit_stream_t stream) {
 }
 
 dit_status dit_selftest_wait_timeout(dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_selftest_wait_timeout");
   const DeviceState* ds = device_state();
   if (!ds || !ds->sm100 || !ds->err) return DIT_ERR_UNSUPPORTED;
   return launch_status(dit::launch_selftest_wait(ds->err, reinterpret_cast<cudaStream_t>(stream)));
@@ -143,6 +159,7 @@ dit_status dit_selftest_wait_timeout(dit_stream_t stream) {
 
 dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, double theta, float* cos_out,
                            float* sin_out, dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_rope_tables");
   if (!pos || !cos_out || !sin_out || N < 1) return DIT_ERR_INVALID_ARG;
   if (d0 < 0 || d1 < 0 || d2 < 0 || (d0 | d1 | d2) & 1 || d0 + d1 + d2 < 2 || d0 + d1 + d2 > 256)
     return DIT_ERR_INVALID_ARG;
@@ -156,6 +173,7 @@ dit_status dit_rope_tables(const int32_t* pos, int N, int d0, int d1, int d2, do
 
 dit_status rope_apply(const void* x, void* y, int B, int H, int N, int d, const int64_t sx[3], const int64_t sy[3],
                       const float* cos_tab, const float* sin_tab, int dtype, dit_stream_t stream) {
+  const NvtxRange nvtx_range("rope_apply");
   if (!x || !y || !sx || !sy || !cos_tab || !sin_tab) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || (dtype != 0 && dtype != 1)) return DIT_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return DIT_ERR_UNSUPPORTED;
@@ -249,6 +267,7 @@ dit_status dit_attn_bf16(const void* q, const void* k, const void* v, void* o, i
                          const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
                          const float* rope_cos, const float* rope_sin, float softmax_scale, void* workspace,
                          size_t workspace_bytes, dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_attn_bf16");
   return attn_bf16_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, workspace,
                         workspace_bytes, nullptr, stream);
 }
@@ -258,6 +277,7 @@ dit_status dit_attn_bf16_skippable(const void* q, const void* k, const void* v, 
                                    const int64_t so[3], const float* rope_cos, const float* rope_sin,
                                    float softmax_scale, void* workspace, size_t workspace_bytes,
                                    const int32_t* skip, dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_attn_bf16_skippable");
   if (!skip) return DIT_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(skip) & 3u) return DIT_ERR_ALIGNMENT;
   return attn_bf16_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, workspace,
@@ -352,6 +372,7 @@ dit_status dit_attn_fp8(const void* q, const void* k, const void* v, void* o, in
                         const int64_t sq[3], const int64_t sk[3], const int64_t sv[3], const int64_t so[3],
                         const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block, int kv_block,
                         int smooth_k, void* workspace, size_t workspace_bytes, dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_attn_fp8");
   return attn_fp8_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, q_block, kv_block,
                        smooth_k, workspace, workspace_bytes, 0, stream);
 }
@@ -361,6 +382,7 @@ dit_status dit_attn_fp8_i8qk(const void* q, const void* k, const void* v, void* 
                              const float* rope_cos, const float* rope_sin, float softmax_scale, int q_block,
                              int kv_block, int smooth_k, void* workspace, size_t workspace_bytes,
                              dit_stream_t stream) {
+  const NvtxRange nvtx_range("dit_attn_fp8_i8qk");
   return attn_fp8_impl(q, k, v, o, B, H, N, d, sq, sk, sv, so, rope_cos, rope_sin, softmax_scale, q_block, kv_block,
                        smooth_k, workspace, workspace_bytes, 1, stream);
 }
@@ -372,6 +394,7 @@ size_t fbcache_gate_workspace_bytes(int64_t n) {
 
 dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float threshold, float* rel_out,
                         int32_t* skip_out, void* workspace, size_t workspace_bytes, dit_stream_t stream) {
+  const NvtxRange nvtx_range("fbcache_gate");
   if (!r_cur || !r_prev || !rel_out || !skip_out || n < 1) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
   if (!aligned16(r_cur) || !aligned16(r_prev) || !aligned4(rel_out) || !aligned4(skip_out)) return DIT_ERR_ALIGNMENT;
@@ -385,6 +408,7 @@ dit_status fbcache_gate(const void* r_cur, const void* r_prev, int64_t n, float 
 
 dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int64_t n, double* sums_out, void* workspace,
                              size_t workspace_bytes, dit_stream_t stream) {
+  const NvtxRange nvtx_range("fbcache_gate_sums");
   if (!r_cur || !r_prev || !sums_out || n < 1) return DIT_ERR_INVALID_ARG;
   if (!aligned16(r_cur) || !aligned16(r_prev) || (reinterpret_cast<uintptr_t>(sums_out) & 7u)) return DIT_ERR_ALIGNMENT;
   const size_t need = fbcache_gate_workspace_bytes(n);
@@ -397,6 +421,7 @@ dit_status fbcache_gate_sums(const void* r_cur, const void* r_prev, int64_t n, d
 
 dit_status fbcache_gate_ref_update(const void* r_cur, void* r_ref, int64_t n, const int32_t* skip,
                                    dit_stream_t stream) {
+  const NvtxRange nvtx_range("fbcache_gate_ref_update");
   if (!r_cur || !r_ref || n < 1) return DIT_ERR_INVALID_ARG;
   if (!aligned16(r_cur) || !aligned16(r_ref) || !aligned4(skip)) return DIT_ERR_ALIGNMENT;
   if (r_cur == r_ref) return DIT_ERR_INVALID_ARG;
@@ -407,6 +432,7 @@ dit_status fbcache_gate_ref_update(const void* r_cur, void* r_ref, int64_t n, co
 
 dit_status fbcache_gate_finalize(const double* sums, float threshold, float* rel_out, int32_t* skip_out,
                                  dit_stream_t stream) {
+  const NvtxRange nvtx_range("fbcache_gate_finalize");
   if (!sums || !rel_out || !skip_out) return DIT_ERR_INVALID_ARG;
   if (!std::isfinite(threshold)) return DIT_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(sums) & 7u) || !aligned4(rel_out) || !aligned4(skip_out)) return DIT_ERR_ALIGNMENT;
