@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(128) kmean_finalize(Fp8Prep p, const float* __
 // through the heads one after another.  Tiles and the rotary rows they need are
 // staged in shared memory by bulk copies issued ahead of use, so the reads
 // never wait on registers: three 32 KB tile slots (one per tensor; a slot is
-// refilled for the next item as soon as every thread has read it) and two
+// refilled for the next item as soon as the 16 converting warps release it) and two
 // 64 KB table slots (cos and sin rows of 128 tokens, one per item in flight,
 // refilled two items ahead).  A producer warp issues the copies as slots are
 // released; sixteen warps convert a tile while the copies of the following
@@ -225,7 +225,7 @@ __device__ __forceinline__ QzItem qz_item(const Fp8Prep& p, int item, int nq) {
 }
 
 __device__ __forceinline__ const __nv_bfloat16* qz_slab(const Fp8Prep& p, int kind, int bh) {
-  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const int b = bh / p.H, h = bh - b * p.H;
   const void* base = kind == kQzQ ? p.q : kind == kQzK ? p.k : p.v;
   const int64_t* s = kind == kQzQ ? p.sq : kind == kQzK ? p.sk : p.sv;
   return static_cast<const __nv_bfloat16*>(base) + b * s[0] + h * s[1];
@@ -489,18 +489,19 @@ __global__ void __launch_bounds__(kQzBlock, 1) quantize_qkv(Fp8Prep p) {
 }  // namespace
 
 cudaError_t launch_fp8_prologue(const Fp8Prep& p, cudaStream_t stream) {
-  float* partial = p.k_partial;
-  dim3 g1(kChunks, p.B * p.H);
-  kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = launch_dependent(kmean_finalize, dim3(p.B * p.H), dim3(128), 0, stream, p, static_cast<const float*>(partial));
-  if (e != cudaSuccess) return e;
+  // every check before the first launch, so that an error return leaves nothing enqueued
   const int64_t items = static_cast<int64_t>(p.B) * p.H * ((p.N + 127) / 128);
   if (items > 0x7fffffff || p.num_sms < 1) return cudaErrorInvalidValue;
   const int grid = static_cast<int>(items < p.num_sms ? items : p.num_sms);  // persistent: one CTA per SM
   auto kern = p.qk_int8 ? quantize_qkv<true> : quantize_qkv<false>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQzSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQzSmem);
+  if (e != cudaSuccess) return e;
+  float* partial = p.k_partial;
+  dim3 g1(kChunks, p.B * p.H);
+  kmean_partial<<<g1, kThreads, 0, stream>>>(p, partial);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(kmean_finalize, dim3(p.B * p.H), dim3(128), 0, stream, p, static_cast<const float*>(partial));
   if (e != cudaSuccess) return e;
   return launch_dependent(kern, dim3(grid), dim3(kQzBlock), kQzSmem, stream, p);
 }
