@@ -329,3 +329,27 @@ def test_planted_drain_only_after_own_failure_is_caught():
             if any(not c[2] for c in s.inflight):
                 caught = True
     assert caught
+
+
+def test_model_matches_the_kernel_source():
+    """The model's shape is the kernel's: 16 converting warps (512 threads), three
+    tile slots and two table slots, full barriers with one arrival and empty
+    barriers with one arrival per converting warp, tiles in the order Q, V, K."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "diffusion_transformer_denoising_dit_b200", "csrc", "fp8_prologue.cu")).read()
+    assert int(re.search(r"constexpr int kQzThreads = (\d+);", src).group(1)) == 32 * WARPS
+    assert "constexpr int kQzBarOff = 3 * kTileBytes + 2 * kTabBytes;" in src
+    kern = src[src.index("quantize_qkv(Fp8Prep p)"):]
+    assert "for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);" in kern            # tile_full[3], tab_full[2]
+    assert "for (int i = 5; i < 10; ++i) mbar_init(&bars[i], kQzThreads / 32);" in kern  # the empties
+    order = [kern.index(f"qz_tile<kQz{k}, INT8>") for k in KINDS]
+    assert order == sorted(order)
+    # the producer stages the table of item n after item n - 2 released it, and
+    # each tile of item n after item n - 1 released that slot; it drains on every exit
+    assert "static_cast<uint32_t>((n - 2) >> 1) & 1u" in kern
+    assert "static_cast<uint32_t>(n - 1) & 1u" in kern
+    producer = kern[kern.index("if (threadIdx.x >= kQzThreads) {"):kern.index("    return;\n  }")]
+    guard = producer[:producer.index("mbar_wait_until")].rsplit("\n    if (", 1)[1].split("\n", 1)[0]
+    assert guard == "(threadIdx.x & 31) == 0) {", guard  # no "!ok": the drain runs whichever way the loop ended
