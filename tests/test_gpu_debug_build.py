@@ -50,6 +50,11 @@ for N in (1, 129, 777):
 for prec in ("fp8", "fp8_i8qk"):
     for N in (1, 65, 700):
         attn(flux, N, prec, 0.995)
+    # no rotary tables: the quantiser stages no table rows
+    q, k, v = synth.qkv(flux, device="cuda", N=300, seed=300)
+    o = dit.attention(q, k, v, None, None, precision=prec).cpu().double().numpy()
+    assert dit.read_error() == 0, ("no rope", prec)
+    assert cos(o, A.attention(q.cpu(), k.cpu(), v.cpu())) >= 0.995, ("no rope", prec)
 cur, prev = synth.gate_pair(2049, 1, 1e-2, device="cuda")
 rel, skip = dit.fbcache_gate(cur, prev, 0.05)
 assert abs(rel.item() - G.relative_l1(cur.cpu(), prev.cpu())) <= 1e-6 * rel.item()

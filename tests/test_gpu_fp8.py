@@ -106,9 +106,13 @@ def test_prologue_matches_oracle_quantiser(precision, N):
     kr = R.apply(k.cpu().double().numpy(), pos, w.axes)
     mean = kr.mean(axis=2)
     np.testing.assert_allclose(views["k_mean"].cpu().numpy(), mean, rtol=1e-4, atol=1e-4)
-    ks = F.smooth_k(kr)
+    _check_codes(views, precision, qr, F.smooth_k(kr), v.cpu().double().numpy())
+
+
+def _check_codes(views, precision, q, k_smoothed, v):
+    """The prologue's codes and scales against the oracle's quantisers."""
     int8 = precision == "fp8_i8qk"
-    for name, x, blk in (("q", qr, 128), ("k", ks, 64), ("v", v.cpu().double().numpy(), 64)):
+    for name, x, blk in (("q", q, 128), ("k", k_smoothed, 64), ("v", v, 64)):
         if int8 and name != "v":
             codes, sc = F.quantize_int8_blocks(x, blk)
             got = views[name + "8"].cpu().view(torch.int8).double().numpy()
@@ -124,6 +128,31 @@ def test_prologue_matches_oracle_quantiser(precision, N):
             assert (rel <= 0.126).all()
         np.testing.assert_allclose(views[name + "_scale"].cpu().double().numpy(), sc, rtol=2e-5)
     np.testing.assert_allclose(views["v_scale_max"].cpu().numpy(), views["v_scale"].cpu().numpy().max(axis=2))
+
+
+@pytest.mark.parametrize("precision", ["fp8", "fp8_i8qk"])
+def test_fp8_without_rotary_tables(precision):
+    """No rotary tables: the prologue stages no table rows and quantises Q and K
+    as given (K still smoothed).  Its codes against the oracle's quantisers on the
+    unrotated inputs; the call against the model of the kernel's arithmetic on
+    those codes and against exact attention without rotation (B = 2, H = 2,
+    N = 700: a ragged last tile)."""
+    w = dataclasses.replace(synth.WORKLOADS["flux1k"], H=2, outliers=False)
+    q, k, v = synth.qkv(w, device=DEV, N=700, B=2, seed=53)
+    B, H, N, d = q.shape
+    ws = dit.attention_workspace(B, H, N, d, precision=precision, device=DEV)
+    o = dit.attention(q, k, v, None, None, precision=precision, workspace=ws)
+    assert dit.read_error() == 0
+    views = dit.fp8_workspace_views(ws, B, H, N, d)
+    kd = k.cpu().double().numpy()
+    np.testing.assert_allclose(views["k_mean"].cpu().numpy(), kd.mean(axis=2), rtol=1e-4, atol=1e-4)
+    _check_codes(views, precision, q.cpu().double().numpy(), F.smooth_k(kd), v.cpu().double().numpy())
+    rows = np.arange(N)
+    exact = A.attention(q.cpu(), k.cpu(), v.cpu())
+    mod = _model_on_kernel_codes(ws, q.shape, precision, rows)
+    o = o.cpu().double().numpy()
+    assert _cos(o, mod) >= MODEL_COS, _cos(o, mod)
+    assert _cos(o, exact) >= TARGET_COS, _cos(o, exact)
 
 
 @pytest.mark.parametrize("precision", ["fp8", "fp8_i8qk"])
